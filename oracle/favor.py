@@ -1,0 +1,212 @@
+"""Plain fp64 CPU restatement of FAVOR+ attention (the oracle).
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module.  It shares no code with ``linear_approximate_softmax_b200/``; the two
+meet only through the seeded inputs that the tests hand to both.
+
+What it computes follows "Rethinking Attention with Performers" (review page):
+the Abstract and section 제안 방법 (proposed method) say that FAVOR+ estimates
+the softmax attention kernel with *positive* *orthogonal* random features, in
+linear time and space, and that the estimate is unbiased; section 주요 결과
+(main results) says orthogonal and positive features lower the mean squared
+error.  The pages do not print the formulas; the reading taken here is the
+plainest one that those statements support:
+
+* x' = d**-0.25 * x for queries and keys, so that exp(q'.k') = exp(q.k/sqrt(d))
+  is the softmax kernel at the usual temperature;
+* phi(x') = exp(W x' - |x'|^2 / 2) / sqrt(m) with W an m x d matrix of random
+  rows, so that E_w[phi(q')^T phi(k')] * m / m = exp(q'.k') (unbiasedness);
+* W: rows drawn N(0, I_d), orthogonalised in blocks of d rows (Gram-Schmidt,
+  fp64, each projection applied twice), then each row rescaled to the length
+  of an independent N(0, I_d) draw (a chi(d) norm), so every row is still
+  marginally N(0, I_d); ``orthogonal=False`` keeps the raw iid rows;
+* out = phi(Q') (phi(K')^T [V | 1]) / last column, never forming L x L
+  (Abstract: linear space and time);
+* stabilisers: one constant per (batch, kv-head) subtracted from every key
+  exponent and one per query row subtracted from that row's exponents.  Both
+  cancel exactly in the ratio; they only keep exp() in range.
+* multi-query layout ("Fast Transformer Decoding: One Write-Head is All You
+  Need", 提出的方法 / proposed method): H query heads share Hkv key/value heads;
+  query head h reads kv head h // (H / Hkv).
+
+Everything is fp64 and written step by step; numpy's matmul, exp and max are
+the only library primitives used.
+"""
+import math
+
+import numpy as np
+
+from . import philox
+
+TAG_DIRECTIONS = 0   # stream of the Gaussian rows that are orthogonalised
+TAG_NORMS = 1        # stream of the Gaussian vectors whose lengths become row norms
+
+
+# --------------------------------------------------------------------------
+# Random features W  ("Rethinking Attention with Performers", Abstract and
+# 제안 방법: positive orthogonal random features)
+# --------------------------------------------------------------------------
+def gram_schmidt_rows(G):
+    """Orthonormalise the rows of a square fp64 matrix, first row first.
+
+    Row i loses its components along rows 0..i-1 (all coefficients taken from
+    the same vector, then subtracted), done twice so the result stays
+    orthogonal to rounding level, and is then scaled to unit length.
+    """
+    G = np.asarray(G, dtype=np.float64)
+    n = G.shape[0]
+    Qm = np.zeros_like(G)
+    for i in range(n):
+        v = G[i].copy()
+        for _ in range(2):
+            if i:
+                coef = Qm[:i] @ v
+                v = v - Qm[:i].T @ coef
+        Qm[i] = v / math.sqrt(float(v @ v))
+    return Qm
+
+
+def make_features(seed, m, d, orthogonal=True):
+    """The m x d random-feature matrix W in fp64 (before storage rounding).
+
+    orthogonal: ceil(m/d) independent d x d Gaussian blocks, each
+    orthonormalised by rows; the first m rows of the stacked blocks are kept
+    and row r is scaled to |h_r| for an independent h_r ~ N(0, I_d).
+    iid: the first m rows of the same Gaussian stream, unchanged.
+    """
+    nblk = (m + d - 1) // d
+    g = philox.normals(seed, TAG_DIRECTIONS, nblk * d * d).reshape(nblk, d, d)
+    if not orthogonal:
+        return g.reshape(nblk * d, d)[:m].copy()
+    dirs = np.concatenate([gram_schmidt_rows(g[b]) for b in range(nblk)], axis=0)[:m]
+    h = philox.normals(seed, TAG_NORMS, m * d).reshape(m, d)
+    norms = np.sqrt(np.sum(h * h, axis=1))
+    return dirs * norms[:, None]
+
+
+def make_features_f32(seed, m, d, orthogonal=True):
+    """W as the library stores it: the fp64 matrix rounded to fp32."""
+    return make_features(seed, m, d, orthogonal).astype(np.float32)
+
+
+# --------------------------------------------------------------------------
+# Feature map and the linear-time estimate (Abstract: linear space and time)
+# --------------------------------------------------------------------------
+def scale_inputs(X):
+    """x' = d**-1/4 x, so that q'.k' = q.k / sqrt(d)."""
+    X = np.asarray(X, dtype=np.float64)
+    return X * X.shape[-1] ** -0.25
+
+
+def exponents(Xs, W):
+    """Rows of W x' - |x'|^2/2 for every scaled row x' of Xs ([n, m])."""
+    W = np.asarray(W, dtype=np.float64)
+    return Xs @ W.T - 0.5 * np.sum(Xs * Xs, axis=1, keepdims=True)
+
+
+def key_features(K, W, stabilise=True):
+    """phi(K') for one kv head, and the key stabiliser that was subtracted.
+
+    The key stabiliser is one constant, the largest exponent of the head, so
+    that every key feature is at most 1/sqrt(m).
+    """
+    m = W.shape[0]
+    u = exponents(scale_inputs(K), W)
+    c = float(u.max()) if stabilise else 0.0
+    return np.exp(u - c) / math.sqrt(m), c
+
+
+def query_features(Q, W, stabilise=True):
+    """phi(Q') for one query head; each row has its own stabiliser (its max)."""
+    m = W.shape[0]
+    u = exponents(scale_inputs(Q), W)
+    c = u.max(axis=1, keepdims=True) if stabilise else np.zeros((u.shape[0], 1))
+    return np.exp(u - c) / math.sqrt(m), c
+
+
+def key_state(K, V, W, stabilise=True):
+    """S = phi(K')^T [V | 1], an m x (d+1) matrix, with its key stabiliser."""
+    phik, c = key_features(K, W, stabilise)
+    V = np.asarray(V, dtype=np.float64)
+    V1 = np.concatenate([V, np.ones((V.shape[0], 1))], axis=1)
+    return phik.T @ V1, c
+
+
+def query_output(Q, W, S, stabilise=True):
+    """out_i = (phi(q_i')^T S[:, :d]) / (phi(q_i')^T S[:, d])."""
+    phiq, _ = query_features(Q, W, stabilise)
+    nz = phiq @ S
+    d = S.shape[1] - 1
+    return nz[:, :d] / nz[:, d:d + 1]
+
+
+def favor_attention(Q, K, V, W, stabilise=True):
+    """FAVOR+ bidirectional attention, fp64.
+
+    Q: [B, H, L, d]; K, V: [B, Hkv, Lk, d]; W: [m, d].  H % Hkv == 0 and
+    query head h reads kv head h // (H // Hkv).  Returns [B, H, L, d] fp64.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, L, d = Q.shape
+    Hkv = K.shape[1]
+    assert H % Hkv == 0
+    G = H // Hkv
+    out = np.empty((B, H, L, d), dtype=np.float64)
+    for b in range(B):
+        for g in range(Hkv):
+            S, _ = key_state(K[b, g], V[b, g], W, stabilise)
+            for h in range(g * G, (g + 1) * G):
+                out[b, h] = query_output(Q[b, h], W, S, stabilise)
+    return out
+
+
+def favor_quadratic(Q, K, V, W):
+    """The same estimate with the L x L matrix formed: D^-1 (phi(Q') phi(K')^T) V.
+
+    Only for tiny L; it checks that the linear-time order of products in
+    ``favor_attention`` changes nothing but rounding.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, L, d = Q.shape
+    G = H // K.shape[1]
+    out = np.empty((B, H, L, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            phiq, _ = query_features(Q[b, h], W)
+            phik, _ = key_features(K[b, h // G], W)
+            A = phiq @ phik.T
+            out[b, h] = (A @ V[b, h // G]) / A.sum(axis=1, keepdims=True)
+    return out
+
+
+def softmax_attention(Q, K, V):
+    """Exact softmax(Q K^T / sqrt(d)) V in fp64, the quantity FAVOR+ estimates."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, L, d = Q.shape
+    G = H // K.shape[1]
+    out = np.empty((B, H, L, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            s = Q[b, h] @ K[b, h // G].T / math.sqrt(d)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            out[b, h] = (p @ V[b, h // G]) / p.sum(axis=1, keepdims=True)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Error metrics used by every parity test
+# --------------------------------------------------------------------------
+def error_metrics(got, ref):
+    """max |got - ref| and sum |got - ref| / sum |ref| (the mean relative error)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    diff = np.abs(got - ref)
+    return float(diff.max()) if diff.size else 0.0, float(diff.sum() / max(np.abs(ref).sum(), 1e-300))

@@ -1,0 +1,138 @@
+"""Pins for the oracle's FAVOR+ estimate.
+
+"Rethinking Attention with Performers" states (Abstract; 주요 결과 / main
+results) that the estimate is unbiased, converges to softmax attention and
+costs linear space and time.  "Fast Transformer Decoding: One Write-Head is
+All You Need" (提出的方法 / proposed method) fixes the shared K/V layout.  Each
+test below checks one of those statements against mathematics or a library
+routine, not against the oracle itself.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import favor
+
+
+def _inputs(B, H, Hkv, L, d, scale=1.0, seed=0):
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((B, H, L, d)) * scale
+    K = rng.standard_normal((B, Hkv, L, d)) * scale
+    V = rng.standard_normal((B, Hkv, L, d))
+    return Q, K, V
+
+
+def test_softmax_attention_matches_torch_sdpa_with_shared_kv():
+    Q, K, V = _inputs(2, 6, 2, 33, 16, seed=1)
+    G = 3
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q), torch.from_numpy(K).repeat_interleave(G, dim=1),
+        torch.from_numpy(V).repeat_interleave(G, dim=1)).numpy()
+    np.testing.assert_allclose(favor.softmax_attention(Q, K, V), want, rtol=1e-10, atol=1e-12)
+
+
+def _mc_kernel_estimates(q, k, d, orthogonal, nseeds):
+    """phi(q')^T phi(k') for m = d features, one W per seed (no stabiliser).
+
+    Each phi carries 1/sqrt(m), so the product is (1/m) sum_r of the
+    per-feature products, the estimator of exp(q.k / sqrt(d)).
+    """
+    est = np.empty(nseeds)
+    for s in range(nseeds):
+        W = favor.make_features(10_000 + s, d, d, orthogonal)
+        pq, _ = favor.query_features(q[None, :], W, stabilise=False)
+        pk, _ = favor.key_features(k[None, :], W, stabilise=False)
+        est[s] = float(pq[0] @ pk[0])
+    return est
+
+
+@pytest.mark.parametrize("orthogonal", [True, False])
+def test_feature_product_is_unbiased_for_softmax_kernel(orthogonal):
+    d = 16
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal(d) * 0.45
+    k = rng.standard_normal(d) * 0.45
+    est = _mc_kernel_estimates(q, k, d, orthogonal, 2000)
+    target = math.exp(float(q @ k) / math.sqrt(d))
+    se = est.std(ddof=1) / math.sqrt(est.size)
+    assert abs(est.mean() - target) < 3.5 * se, (est.mean(), target, se)
+    assert se < 0.05 * target  # the check has teeth
+
+
+def test_orthogonal_features_lower_the_variance():
+    # 주요 결과: orthogonal random features reduce the mean squared error
+    d = 16
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal(d) * 0.3
+    k = rng.standard_normal(d) * 0.3
+    target = math.exp(float(q @ k) / math.sqrt(d))
+    n = 4000
+    e_orf = (_mc_kernel_estimates(q, k, d, True, n) - target) ** 2
+    e_iid = (_mc_kernel_estimates(q, k, d, False, n) - target) ** 2
+    se = math.sqrt(e_orf.var() / n + e_iid.var() / n)
+    assert e_iid.mean() - e_orf.mean() > 2.0 * se, (e_orf.mean(), e_iid.mean(), se)
+
+
+def test_linear_order_equals_quadratic_form():
+    Q, K, V = _inputs(1, 4, 2, 40, 16, scale=0.7, seed=2)
+    W = favor.make_features(3, 48, 16)
+    lin = favor.favor_attention(Q, K, V, W)
+    quad = favor.favor_quadratic(Q, K, V, W)
+    np.testing.assert_allclose(lin, quad, rtol=1e-12, atol=1e-13)
+
+
+def test_stabilisers_cancel_exactly():
+    Q, K, V = _inputs(2, 2, 1, 50, 16, scale=0.8, seed=3)
+    W = favor.make_features(4, 64, 16)
+    a = favor.favor_attention(Q, K, V, W, stabilise=True)
+    b = favor.favor_attention(Q, K, V, W, stabilise=False)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+
+
+def test_stabilisers_keep_large_inputs_finite():
+    # exponents near -900: without the stabiliser exp() underflows to 0 and the ratio is 0/0
+    Q, K, V = _inputs(1, 1, 1, 20, 16, scale=25.0, seed=4)
+    W = favor.make_features(5, 32, 16)
+    out = favor.favor_attention(Q, K, V, W)
+    assert np.all(np.isfinite(out))
+    with np.errstate(invalid="ignore", divide="ignore"):
+        raw = favor.favor_attention(Q, K, V, W, stabilise=False)
+    assert not np.all(np.isfinite(raw))
+
+
+def test_outputs_are_convex_combinations_of_values():
+    Q, K, V = _inputs(2, 4, 2, 64, 16, seed=5)
+    W = favor.make_features(6, 32, 16)
+    out = favor.favor_attention(Q, K, V, W)
+    G = 2
+    for b in range(2):
+        for h in range(4):
+            lo = V[b, h // G].min(axis=0)
+            hi = V[b, h // G].max(axis=0)
+            assert np.all(out[b, h] >= lo - 1e-12) and np.all(out[b, h] <= hi + 1e-12)
+
+
+def test_converges_to_softmax_attention_as_m_grows():
+    # small-norm inputs (Q, K ~ N(0, 0.25^2)); shared K/V heads included
+    d, L = 16, 16
+    rng = np.random.default_rng(12)
+    Q = rng.standard_normal((1, 4, L, d)) * 0.25
+    K = rng.standard_normal((1, 2, L, d)) * 0.25
+    V = rng.standard_normal((1, 2, L, d))
+    exact = favor.softmax_attention(Q, K, V)
+    errs = []
+    for m in (16, 256, 4096, 16384):
+        e = [np.abs(favor.favor_attention(Q, K, V, favor.make_features(s, m, d)) - exact).max()
+             for s in range(20)]
+        errs.append(float(np.mean(e)))
+    assert all(a > b for a, b in zip(errs, errs[1:])), errs
+    assert errs[-1] <= 1e-2, errs
+
+
+def test_error_metrics():
+    ref = np.array([1.0, -2.0, 0.0, 1.0])
+    got = np.array([1.5, -2.0, 0.25, 1.0])
+    ma, mr = favor.error_metrics(got, ref)
+    assert ma == 0.5 and mr == pytest.approx(0.75 / 4.0)
