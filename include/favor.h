@@ -1,0 +1,165 @@
+/*
+ * favor.h — C ABI of the B200 (sm_100a) FAVOR+ attention library.
+ *
+ * FAVOR+ ("Rethinking Attention with Performers", Abstract and section
+ * 제안 방법 / proposed method) estimates softmax attention with positive
+ * orthogonal random features in time and memory linear in the sequence length:
+ *
+ *   x'      = d^(-1/4) x                     (queries and keys)
+ *   phi(x') = exp(W x' - |x'|^2/2) / sqrt(m) (W: m x d random features)
+ *   out     = phi(Q') (phi(K')^T [V | 1]) / (last column)
+ *
+ * and the L x L attention matrix is never formed.  Query head h reads key/value
+ * head h / (H / Hkv): the multi-query layout of "Fast Transformer Decoding:
+ * One Write-Head is All You Need" (提出的方法 / proposed method) when Hkv = 1.
+ *
+ * Conventions shared by every entry point:
+ *  - Return 0 (FAVOR_OK) on success, a negative FAVOR_ERR_* code on failure;
+ *    favor_last_error() then holds a message (thread-local).  Nothing throws
+ *    across the ABI and no argument error launches any GPU work.
+ *  - Tensors are dense, contiguous, row-major:
+ *      Q, out [B, H, L, d];  K, V [B, Hkv, L, d];  W [m, d] fp32.
+ *  - Device pointers must be 16-byte aligned (FAVOR_ERR_INVALID otherwise).
+ *  - The caller owns every buffer it passes; the library keeps no pointer to
+ *    any of them after a call returns.
+ *  - GPU entry points are asynchronous on `stream` (0 = legacy default
+ *    stream) and never synchronise it; CUDA launch errors are reported as
+ *    FAVOR_ERR_CUDA.
+ *  - Supported shapes: d in {64, 128}; m a multiple of 16 with 16 <= m <= 512;
+ *    B, H, Hkv, L >= 1; H % Hkv == 0.  Anything else is FAVOR_ERR_UNSUPPORTED.
+ */
+#ifndef FAVOR_B200_H
+#define FAVOR_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* favor_stream_t; /* the same type as cudaStream_t */
+
+#if defined(__GNUC__)
+#define FAVOR_API __attribute__((visibility("default")))
+#else
+#define FAVOR_API
+#endif
+
+#define FAVOR_OK 0
+#define FAVOR_ERR_INVALID (-1)     /* null or misaligned pointer, bad size or flag   */
+#define FAVOR_ERR_UNSUPPORTED (-2) /* shape outside the supported set (see above)     */
+#define FAVOR_ERR_CUDA (-3)        /* a CUDA runtime call or launch failed            */
+#define FAVOR_ERR_NOMEM (-4)       /* a host or device allocation failed              */
+
+/* Element type of Q, K, V and out. */
+#define FAVOR_BF16 0
+#define FAVOR_F32 1
+
+/* Message for the last non-zero return on the calling thread ("" if none). */
+FAVOR_API const char* favor_last_error(void);
+
+/* Library version, e.g. 100 for 0.1.0. */
+FAVOR_API int favor_version(void);
+
+/*
+ * favor_make_features — the random-feature matrix W (host only, no GPU).
+ *
+ * "Rethinking Attention with Performers", Abstract / 제안 방법: positive
+ * orthogonal random features.  orthogonal != 0: ceil(m/d) independent d x d
+ * blocks of standard normals, rows orthonormalised first to last by
+ * Gram-Schmidt in fp64 (each projection applied twice); the first m rows of
+ * the stacked blocks are kept and row r is scaled to the length |h_r| of an
+ * independent h_r ~ N(0, I_d), so every row is marginally N(0, I_d).
+ * orthogonal == 0: the first m rows of the same normal stream, unchanged.
+ *
+ * Random numbers: Philox4x64-10 (Salmon et al., SC'11) with key (seed, 0);
+ * the n-th normal of stream t comes from counter (n/4, t, 0, 0) through
+ * Box-Muller on u = ((x >> 12) + 1/2) 2^-52.  Stream 0 feeds the blocks,
+ * stream 1 the norm vectors.  The same (seed, m, d, orthogonal) always gives
+ * the same W, on any machine, up to the last bit of the fp64 libm.
+ *
+ * W_out: host, caller-owned, m*d floats, row-major [m, d], written as the fp64
+ * result rounded to fp32.  W is passed to the attention calls UNSCALED.
+ * Errors: FAVOR_ERR_INVALID (null W_out, m < 1, d < 1),
+ * FAVOR_ERR_NOMEM (scratch allocation failed).  Any m, d >= 1 is accepted.
+ */
+FAVOR_API int favor_make_features(uint64_t seed, int m, int d, int orthogonal, float* W_out);
+
+/*
+ * favor_attention — bf16 FAVOR+ attention, bidirectional (device pointers).
+ *
+ * Q [B,H,L,d], K and V [B,Hkv,L,d] bf16; W [m,d] fp32 (unscaled, as
+ * favor_make_features writes it); out [B,H,L,d] bf16.  Accumulation is fp32.
+ * The path: key pass (phi(K') and per-chunk partial states phi(K')^T [V|1],
+ * each with its own max stabiliser), a fixed-order reduction that rescales the
+ * partials to one stabiliser (bitwise deterministic), then the query pass
+ * (phi(Q') with a per-row stabiliser, the product with the state, and the
+ * division by the last column).  The scratch memory it needs (partials and
+ * the state) is allocated and freed stream-ordered on `stream`
+ * (cudaMallocAsync / cudaFreeAsync); FAVOR_ERR_CUDA if that fails.
+ */
+FAVOR_API int favor_attention(const void* Q, const void* K, const void* V, const float* W, void* out,
+                    int B, int H, int Hkv, int L, int d, int m, favor_stream_t stream);
+
+/* favor_attention_f32 — the same with fp32 Q, K, V and out (fp32 arithmetic
+ * throughout, no tensor-core rounding). */
+FAVOR_API int favor_attention_f32(const float* Q, const float* K, const float* V, const float* W, float* out,
+                        int B, int H, int Hkv, int L, int d, int m, favor_stream_t stream);
+
+/*
+ * favor_attention_host — end-to-end call on HOST buffers.
+ *
+ * Q, K, V, out are host pointers (pinned memory gives asynchronous copies;
+ * pageable memory works, slower); W is a host [m,d] fp32 array.  dtype is
+ * FAVOR_BF16 or FAVOR_F32 for Q, K, V and out.  The call copies the inputs to
+ * the device, runs favor_attention(_f32) on `stream`, copies out back, and
+ * synchronises `stream` before returning.  Device buffers are allocated and
+ * freed stream-ordered inside the call.
+ */
+FAVOR_API int favor_attention_host(int dtype, const void* Q, const void* K, const void* V, const float* W,
+                         void* out, int B, int H, int Hkv, int L, int d, int m,
+                         favor_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Stage-level calls.  favor_attention == favor_key_pass + favor_state_reduce +
+ * favor_query_pass on one stream, with the caller providing the scratch.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of key-pass partials for this shape on the current device (the chunk
+ * count depends on the device's SM count).  0 for unsupported shapes. */
+FAVOR_API size_t favor_partials_bytes(int B, int Hkv, int L, int d, int m);
+
+/*
+ * Bytes of the reduced state for B*Hkv kv heads.  Layout (fp32 unless noted):
+ *   S    [B*Hkv][m][d+1]   phi(K')^T [V | 1] scaled by 2^(-c) (c per kv head)
+ *   c    [B*Hkv]           the key stabiliser, in log2 units
+ *   then an internal region (the state re-packed as tensor-core operands),
+ *   written by favor_state_reduce and read by favor_query_pass.
+ * 0 for unsupported shapes.
+ */
+FAVOR_API size_t favor_state_bytes(int B, int Hkv, int d, int m);
+
+/* favor_key_pass — phi(K') and the partial states of every key chunk.
+ * dtype: FAVOR_BF16 or FAVOR_F32 (element type of K and V).  partials: device,
+ * caller-owned, favor_partials_bytes(...) bytes, fully overwritten. */
+FAVOR_API int favor_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials,
+                   int B, int Hkv, int L, int d, int m, favor_stream_t stream);
+
+/* favor_state_reduce — rescale the partials of each kv head to the largest
+ * chunk stabiliser and sum them in chunk order (bitwise deterministic).
+ * state: device, caller-owned, favor_state_bytes(...) bytes, fully overwritten. */
+FAVOR_API int favor_state_reduce(const void* partials, void* state, int B, int Hkv, int L, int d, int m,
+                       favor_stream_t stream);
+
+/* favor_query_pass — out = phi(Q') S[:, :d] / phi(Q') S[:, d] for every query
+ * head, reading the state of kv head h / (H/Hkv).  dtype as for the key pass
+ * (element type of Q and out). */
+FAVOR_API int favor_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out,
+                     int B, int H, int Hkv, int L, int d, int m, favor_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FAVOR_B200_H */

@@ -1,0 +1,246 @@
+// C ABI of the FAVOR+ library: argument checks, planning, scratch and dispatch.
+// Every exported function is declared and documented in include/favor.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "favor_internal.h"
+
+namespace favor {
+
+namespace {
+thread_local std::string g_last_error;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int H, int Hkv, int L, int d, int m) {
+  if (B < 1 || H < 1 || Hkv < 1 || L < 1)
+    return set_errorf(FAVOR_ERR_UNSUPPORTED, "B, H, Hkv and L must be >= 1 (got %d, %d, %d, %d)", B, H, Hkv, L);
+  if (H % Hkv != 0) return set_errorf(FAVOR_ERR_UNSUPPORTED, "H (%d) must be a multiple of Hkv (%d)", H, Hkv);
+  if (d != 64 && d != 128) return set_errorf(FAVOR_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+  if (m < 16 || m > 512 || m % 16 != 0)
+    return set_errorf(FAVOR_ERR_UNSUPPORTED, "m must be a multiple of 16 in [16, 512] (got %d)", m);
+  const double elems = static_cast<double>(B) * H * L * d;
+  if (elems > 4.0e12) return set_error(FAVOR_ERR_UNSUPPORTED, "tensor too large");
+  return FAVOR_OK;
+}
+
+int check_dtype(int dtype) {
+  if (dtype != FAVOR_BF16 && dtype != FAVOR_F32)
+    return set_errorf(FAVOR_ERR_INVALID, "dtype must be FAVOR_BF16 (0) or FAVOR_F32 (1), got %d", dtype);
+  return FAVOR_OK;
+}
+
+int check_ptrs(const char* what, std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs) {
+    if (!p) return set_errorf(FAVOR_ERR_INVALID, "%s: null pointer argument", what);
+    if (!aligned16(p)) return set_errorf(FAVOR_ERR_INVALID, "%s: pointer %p is not 16-byte aligned", what, p);
+  }
+  return FAVOR_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int device_sm_count(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "no usable CUDA device: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
+#define FAVOR_TRY(expr)            \
+  do {                             \
+    int _rc = (expr);              \
+    if (_rc != FAVOR_OK) return _rc; \
+  } while (0)
+
+#define FAVOR_CUDA_TRY(expr, what)                                                      \
+  do {                                                                                  \
+    cudaError_t _e = (expr);                                                            \
+    if (_e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(_e)); \
+  } while (0)
+
+}  // namespace
+
+int set_error(int code, const char* msg) {
+  g_last_error = msg ? msg : "";
+  return code;
+}
+
+int set_errorf(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
+  FAVOR_TRY(check_shape(B, H, Hkv, L, d, m));
+  int sms = 0;
+  FAVOR_TRY(device_sm_count(&sms));
+  p->B = B; p->H = H; p->Hkv = Hkv; p->L = L; p->d = d; p->m = m;
+  const int heads = B * Hkv;
+  const int tiles = (L + kTileTokens - 1) / kTileTokens;
+  // About two key-pass CTAs per SM for each 64-feature block of every kv head.
+  long want = (2L * sms + heads - 1) / heads;
+  if (want < 1) want = 1;
+  if (want > tiles) want = tiles;
+  const int chunk_tiles = (tiles + static_cast<int>(want) - 1) / static_cast<int>(want);
+  p->chunk = chunk_tiles * kTileTokens;
+  p->P = (tiles + chunk_tiles - 1) / chunk_tiles;
+  p->nsb = (m + kStabBlock - 1) / kStabBlock;
+  const size_t D1 = static_cast<size_t>(d) + 1;
+  p->part_S_off = 0;
+  p->part_c_off = round_up(sizeof(float) * heads * p->P * m * D1, 256);
+  p->part_bytes = p->part_c_off + round_up(sizeof(float) * heads * p->P * p->nsb, 256);
+  p->st_S_off = 0;
+  p->st_c_off = round_up(sizeof(float) * heads * m * D1, 256);
+  p->st_op_off = p->st_c_off + round_up(sizeof(float) * heads, 256);
+  p->st_bytes = p->st_op_off;
+  p->wscale = static_cast<float>(std::pow(static_cast<double>(d), -0.25) * kLog2e);
+  p->nscale = static_cast<float>(std::pow(static_cast<double>(d), -0.5) * kLog2e * 0.5);
+  return FAVOR_OK;
+}
+
+namespace {
+
+int run_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials, const Plan& p,
+                 cudaStream_t st) {
+  return simt_key_pass(dtype, K, V, W, partials, p, st);
+}
+
+int run_reduce(const void* partials, void* state, const Plan& p, cudaStream_t st) {
+  return simt_state_reduce(partials, state, p, st);
+}
+
+int run_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out, const Plan& p,
+                   cudaStream_t st) {
+  return simt_query_pass(dtype, Q, W, state, out, p, st);
+}
+
+int attention_impl(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,
+                   int H, int Hkv, int L, int d, int m, cudaStream_t st) {
+  FAVOR_TRY(check_dtype(dtype));
+  FAVOR_TRY(check_ptrs("favor_attention", {Q, K, V, W, out}));
+  Plan p;
+  FAVOR_TRY(make_plan(B, H, Hkv, L, d, m, &p));
+  void* ws = nullptr;
+  const size_t st_off = round_up(p.part_bytes, 256);
+  FAVOR_CUDA_TRY(cudaMallocAsync(&ws, st_off + p.st_bytes, st), "favor_attention scratch allocation");
+  char* base = static_cast<char*>(ws);
+  int rc = run_key_pass(dtype, K, V, W, base, p, st);
+  if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, p, st);
+  if (rc == FAVOR_OK) rc = run_query_pass(dtype, Q, W, base + st_off, out, p, st);
+  cudaError_t fe = cudaFreeAsync(ws, st);
+  if (rc != FAVOR_OK) return rc;
+  FAVOR_CUDA_TRY(fe, "favor_attention scratch release");
+  return FAVOR_OK;
+}
+
+}  // namespace
+}  // namespace favor
+
+using namespace favor;
+
+extern "C" {
+
+const char* favor_last_error(void) { return g_last_error.c_str(); }
+
+int favor_version(void) { return 100; }
+
+int favor_make_features(uint64_t seed, int m, int d, int orthogonal, float* W_out) {
+  return make_features(seed, m, d, orthogonal, W_out);
+}
+
+int favor_attention(const void* Q, const void* K, const void* V, const float* W, void* out, int B, int H,
+                    int Hkv, int L, int d, int m, favor_stream_t stream) {
+  return attention_impl(FAVOR_BF16, Q, K, V, W, out, B, H, Hkv, L, d, m, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int favor_attention_f32(const float* Q, const float* K, const float* V, const float* W, float* out, int B, int H,
+                        int Hkv, int L, int d, int m, favor_stream_t stream) {
+  return attention_impl(FAVOR_F32, Q, K, V, W, out, B, H, Hkv, L, d, m, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int favor_attention_host(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,
+                         int H, int Hkv, int L, int d, int m, favor_stream_t stream) {
+  FAVOR_TRY(check_dtype(dtype));
+  if (!Q || !K || !V || !W || !out) return set_error(FAVOR_ERR_INVALID, "favor_attention_host: null pointer argument");
+  FAVOR_TRY(check_shape(B, H, Hkv, L, d, m));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = dtype == FAVOR_F32 ? 4 : 2;
+  const size_t nq = static_cast<size_t>(B) * H * L * d, nk = static_cast<size_t>(B) * Hkv * L * d;
+  const size_t bq = round_up(nq * es, 256), bk = round_up(nk * es, 256), bw = round_up(sizeof(float) * m * d, 256);
+  void* buf = nullptr;
+  FAVOR_CUDA_TRY(cudaMallocAsync(&buf, 2 * bq + 2 * bk + bw, st), "favor_attention_host device allocation");
+  char* dQ = static_cast<char*>(buf);
+  char* dK = dQ + bq;
+  char* dV = dK + bk;
+  char* dW = dV + bk;
+  char* dO = dW + bw;
+  int rc = FAVOR_OK;
+  cudaError_t e = cudaMemcpyAsync(dQ, Q, nq * es, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dK, K, nk * es, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dV, V, nk * es, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dW, W, sizeof(float) * m * d, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) rc = set_errorf(FAVOR_ERR_CUDA, "favor_attention_host copy in: %s", cudaGetErrorString(e));
+  if (rc == FAVOR_OK)
+    rc = attention_impl(dtype, dQ, dK, dV, reinterpret_cast<const float*>(dW), dO, B, H, Hkv, L, d, m, st);
+  if (rc == FAVOR_OK) {
+    e = cudaMemcpyAsync(out, dO, nq * es, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) rc = set_errorf(FAVOR_ERR_CUDA, "favor_attention_host copy out: %s", cudaGetErrorString(e));
+  }
+  cudaError_t fe = cudaFreeAsync(buf, st);
+  cudaError_t se = cudaStreamSynchronize(st);
+  if (rc != FAVOR_OK) return rc;
+  if (fe != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "favor_attention_host release: %s", cudaGetErrorString(fe));
+  if (se != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "favor_attention_host: %s", cudaGetErrorString(se));
+  return FAVOR_OK;
+}
+
+size_t favor_partials_bytes(int B, int Hkv, int L, int d, int m) {
+  Plan p;
+  if (make_plan(B, Hkv, Hkv, L, d, m, &p) != FAVOR_OK) return 0;
+  return p.part_bytes;
+}
+
+size_t favor_state_bytes(int B, int Hkv, int d, int m) {
+  Plan p;
+  if (make_plan(B, Hkv, Hkv, 1, d, m, &p) != FAVOR_OK) return 0;
+  return p.st_bytes;
+}
+
+int favor_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials, int B, int Hkv, int L,
+                   int d, int m, favor_stream_t stream) {
+  FAVOR_TRY(check_dtype(dtype));
+  FAVOR_TRY(check_ptrs("favor_key_pass", {K, V, W, partials}));
+  Plan p;
+  FAVOR_TRY(make_plan(B, Hkv, Hkv, L, d, m, &p));
+  return run_key_pass(dtype, K, V, W, partials, p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int favor_state_reduce(const void* partials, void* state, int B, int Hkv, int L, int d, int m,
+                       favor_stream_t stream) {
+  FAVOR_TRY(check_ptrs("favor_state_reduce", {partials, state}));
+  Plan p;
+  FAVOR_TRY(make_plan(B, Hkv, Hkv, L, d, m, &p));
+  return run_reduce(partials, state, p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int favor_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out, int B, int H, int Hkv,
+                     int L, int d, int m, favor_stream_t stream) {
+  FAVOR_TRY(check_dtype(dtype));
+  FAVOR_TRY(check_ptrs("favor_query_pass", {Q, W, state, out}));
+  Plan p;
+  FAVOR_TRY(make_plan(B, H, Hkv, L, d, m, &p));
+  return run_query_pass(dtype, Q, W, state, out, p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Internal declarations shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "favor.h"
+
+namespace favor {
+
+// Records `msg` as the calling thread's last error and returns `code`.
+int set_error(int code, const char* msg);
+int set_errorf(int code, const char* fmt, ...);
+
+int make_features(uint64_t seed, int m, int d, int orthogonal, float* W_out);
+
+constexpr double kLog2e = 1.4426950408889634074;
+constexpr int kTileTokens = 128;   // key chunks are whole multiples of this
+constexpr int kStabBlock = 64;     // partial stabilisers are kept per 64 features
+
+// How the key pass splits each kv head's L tokens into P chunks.
+struct Plan {
+  int B, H, Hkv, L, d, m;
+  int P;            // chunks per kv head
+  int chunk;        // tokens per chunk (multiple of kTileTokens, last one ragged)
+  int nsb;          // stabiliser blocks: ceil(m / kStabBlock)
+  // byte offsets inside the partials buffer
+  size_t part_S_off, part_c_off, part_bytes;
+  // byte offsets inside the state buffer
+  size_t st_S_off, st_c_off, st_op_off, st_bytes;
+  float wscale;     // d^-1/4 * log2(e): W is multiplied by this on the device
+  float nscale;     // d^-1/2 * log2(e) / 2: |k|^2 is multiplied by this
+};
+
+// Fills `p` for a validated shape on the current device.  Returns FAVOR_OK or an error.
+int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p);
+
+// ---- CUDA-core kernels (fp32 arithmetic; fp32 or bf16 storage) -------------
+int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials,
+                  const Plan& p, void* stream);
+int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream);
+int simt_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out,
+                    const Plan& p, void* stream);
+
+}  // namespace favor

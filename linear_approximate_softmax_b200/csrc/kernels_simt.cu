@@ -1,0 +1,324 @@
+// FAVOR+ on CUDA cores: fp32 arithmetic throughout, fp32 or bf16 storage.
+//
+// This is the exact-arithmetic path (the fp32 entry point) and the reference
+// GPU path for bf16 inputs.  Three kernels, one per step of the linear-time
+// estimate ("Rethinking Attention with Performers", Abstract: linear space and
+// time; 제안 방법: positive random features):
+//
+//   key pass     per (kv head, key chunk, 64-feature block):
+//                u = W'k - n(k) (log2 units), chunk max stabiliser c (running,
+//                with exact rescaling of the accumulator when it grows),
+//                S_part = sum_t 2^(u_t - c) [v_t | 1]
+//   reduce       per kv head: c* = max c, S = sum_p 2^(c_p - c*) S_p in chunk order
+//   query pass   per (query head, 32-query tile): u = W'q, per-row max
+//                stabiliser, out = (phi S[:, :d]) / (phi S[:, d])
+//
+// W' = d^-1/4 log2(e) W and n(k) = d^-1/2 log2(e) |k|^2 / 2, so 2^(W'k - n(k))
+// = exp(W k' - |k'|^2/2) with k' = d^-1/4 k.  The query's -|q'|^2/2 term and
+// the 1/sqrt(m) factors are constant along a query row and cancel exactly in
+// the ratio, as any per-row stabiliser does; they are not computed.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "favor_internal.h"
+
+namespace favor {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kFB = 64;   // features per key-pass CTA (== kStabBlock)
+constexpr int kTT = 32;   // tokens per key-pass step
+constexpr int kQT = 32;   // queries per query-pass CTA
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void store_as(float* p, float x) { *p = x; }
+__device__ __forceinline__ void store_as(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// grid (P, B*Hkv, ceil(m/64)), 256 threads.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) key_pass_kernel(
+    const T* __restrict__ K, const T* __restrict__ V, const float* __restrict__ W,
+    float* __restrict__ part_S, float* __restrict__ part_c, int L, int m, int P, int chunk,
+    int nsb, float wscale, float nscale) {
+  constexpr int D1 = D + 1;
+  constexpr int NE = (kFB * D1 + kThreads - 1) / kThreads;
+  extern __shared__ float smem[];
+  float* Ws = smem;                  // [kFB][D1]   (row stride D1 keeps banks apart)
+  float* Ks = Ws + kFB * D1;         // [kTT][D1]   column D holds n(k)
+  float* Vs = Ks + kTT * D1;         // [kTT][D1]   column D holds 1 (0 past the end)
+  float* U = Vs + kTT * D1;          // [kTT][kFB+1]
+  float* red = U + kTT * (kFB + 1);  // [kThreads/32]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int p = blockIdx.x, head = blockIdx.y, fb = blockIdx.z;
+  const int f0 = fb * kFB, fbw = min(kFB, m - f0);
+  const int t_begin = p * chunk, t_end = min(L, t_begin + chunk);
+  const T* Kh = K + static_cast<size_t>(head) * L * D;
+  const T* Vh = V + static_cast<size_t>(head) * L * D;
+
+  for (int i = tid; i < kFB * D; i += kThreads) {
+    const int f = i / D, j = i % D;
+    Ws[f * D1 + j] = f < fbw ? W[static_cast<size_t>(f0 + f) * D + j] * wscale : 0.f;
+  }
+
+  float acc[NE];
+#pragma unroll
+  for (int k = 0; k < NE; ++k) acc[k] = 0.f;
+  float c_run = -INFINITY;
+
+  for (int t0 = t_begin; t0 < t_end; t0 += kTT) {
+    const int tw = min(kTT, t_end - t0);
+    __syncthreads();  // previous step is done with Ks, Vs, U, red
+    for (int i = tid; i < kTT * D; i += kThreads) {
+      const int t = i / D, j = i % D;
+      float kv = 0.f, vv = 0.f;
+      if (t < tw) {
+        kv = to_f32(Kh[static_cast<size_t>(t0 + t) * D + j]);
+        vv = to_f32(Vh[static_cast<size_t>(t0 + t) * D + j]);
+      }
+      Ks[t * D1 + j] = kv;
+      Vs[t * D1 + j] = vv;
+    }
+    if (tid < kTT) Vs[tid * D1 + D] = tid < tw ? 1.f : 0.f;
+    __syncthreads();
+    if (tid < kTT) {
+      float s = 0.f;
+      for (int j = 0; j < D; ++j) s = fmaf(Ks[tid * D1 + j], Ks[tid * D1 + j], s);
+      Ks[tid * D1 + D] = s * nscale;
+    }
+    __syncthreads();
+
+    float lmax = -INFINITY;
+    for (int i = tid; i < kTT * kFB; i += kThreads) {
+      const int t = i / kFB, f = i % kFB;
+      float u = -INFINITY;
+      if (t < tw && f < fbw) {
+        float s = 0.f;
+#pragma unroll 16
+        for (int j = 0; j < D; ++j) s = fmaf(Ks[t * D1 + j], Ws[f * D1 + j], s);
+        u = s - Ks[t * D1 + D];
+      }
+      U[t * (kFB + 1) + f] = u;
+      lmax = fmaxf(lmax, u);
+    }
+    lmax = warp_max(lmax);
+    if (lane == 0) red[warp] = lmax;
+    __syncthreads();
+    float tmax = red[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) tmax = fmaxf(tmax, red[w]);
+    const float c_new = fmaxf(c_run, tmax);
+    const float rescale = (c_run == -INFINITY) ? 1.f : exp2f(c_run - c_new);
+    c_run = c_new;
+    for (int i = tid; i < kTT * kFB; i += kThreads) {
+      const int t = i / kFB, f = i % kFB;
+      const float u = U[t * (kFB + 1) + f];
+      U[t * (kFB + 1) + f] = (u == -INFINITY) ? 0.f : exp2f(u - c_new);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < NE; ++k) {
+      const int e = tid + k * kThreads;
+      if (e < kFB * D1) {
+        const int f = e / D1, c = e % D1;
+        float a = acc[k] * rescale;
+        for (int t = 0; t < tw; ++t) a = fmaf(U[t * (kFB + 1) + f], Vs[t * D1 + c], a);
+        acc[k] = a;
+      }
+    }
+  }
+
+  float* out = part_S + (static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * D1;
+#pragma unroll
+  for (int k = 0; k < NE; ++k) {
+    const int e = tid + k * kThreads;
+    if (e < kFB * D1) {
+      const int f = e / D1, c = e % D1;
+      if (f < fbw) out[static_cast<size_t>(f0 + f) * D1 + c] = acc[k];
+    }
+  }
+  if (tid == 0) part_c[(static_cast<size_t>(head) * P + p) * nsb + fb] = c_run;
+}
+
+// grid (ceil(m*(d+1)/256), B*Hkv), 256 threads.  Fixed summation order p = 0..P-1.
+__global__ void __launch_bounds__(kThreads) state_reduce_kernel(
+    const float* __restrict__ part_S, const float* __restrict__ part_c, float* __restrict__ S,
+    float* __restrict__ Sc, int P, int m, int D1, int nsb) {
+  const int head = blockIdx.y;
+  const int e = blockIdx.x * kThreads + threadIdx.x;
+  const float* pc = part_c + static_cast<size_t>(head) * P * nsb;
+  float cs = -INFINITY;
+  for (int i = 0; i < P * nsb; ++i) cs = fmaxf(cs, pc[i]);
+  if (e < m * D1) {
+    const int sb = (e / D1) / kStabBlock;
+    float s = 0.f;
+    for (int p = 0; p < P; ++p) {
+      const float c = pc[p * nsb + sb];
+      const float w = (c == -INFINITY) ? 0.f : exp2f(c - cs);
+      s = fmaf(w, part_S[(static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * D1 + e], s);
+    }
+    S[static_cast<size_t>(head) * m * D1 + e] = s;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) Sc[head] = cs;
+}
+
+// grid (ceil(L/32), B*H), 256 threads.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) query_pass_kernel(
+    const T* __restrict__ Q, const float* __restrict__ W, const float* __restrict__ S,
+    T* __restrict__ out, int L, int m, int H, int Hkv, float wscale) {
+  constexpr int D1 = D + 1;
+  constexpr int NE = (kQT * D1 + kThreads - 1) / kThreads;
+  extern __shared__ float smem[];
+  const int mp = m + 1;
+  float* Qs = smem;               // [kQT][D1]
+  float* Ws = Qs + kQT * D1;      // [kFB][D1]
+  float* O = Ws + kFB * D1;       // [kQT][D1 + 1]
+  float* U = O + kQT * (D1 + 1);  // [kQT][m + 1]
+
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int kvh = b * Hkv + h / (H / Hkv);
+  const int q0 = blockIdx.x * kQT, qw = min(kQT, L - q0);
+  const T* Qh = Q + static_cast<size_t>(bh) * L * D;
+  const float* Sh = S + static_cast<size_t>(kvh) * m * D1;
+
+  for (int i = tid; i < kQT * D; i += kThreads) {
+    const int r = i / D, j = i % D;
+    Qs[r * D1 + j] = r < qw ? to_f32(Qh[static_cast<size_t>(q0 + r) * D + j]) : 0.f;
+  }
+  for (int f0 = 0; f0 < m; f0 += kFB) {
+    const int fbw = min(kFB, m - f0);
+    __syncthreads();  // Qs ready / previous block done with Ws
+    for (int i = tid; i < kFB * D; i += kThreads) {
+      const int f = i / D, j = i % D;
+      Ws[f * D1 + j] = f < fbw ? W[static_cast<size_t>(f0 + f) * D + j] * wscale : 0.f;
+    }
+    __syncthreads();
+    for (int i = tid; i < kQT * kFB; i += kThreads) {
+      const int r = i / kFB, f = i % kFB;
+      if (f < fbw) {
+        float s = 0.f;
+#pragma unroll 16
+        for (int j = 0; j < D; ++j) s = fmaf(Qs[r * D1 + j], Ws[f * D1 + j], s);
+        U[r * mp + f0 + f] = s;
+      }
+    }
+  }
+  __syncthreads();
+  {  // per-row max over the m features, then phi in place; 8 threads per row
+    const int r = tid >> 3, k = tid & 7;
+    float mx = -INFINITY;
+    for (int f = k; f < m; f += 8) mx = fmaxf(mx, U[r * mp + f]);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    for (int f = k; f < m; f += 8) U[r * mp + f] = exp2f(U[r * mp + f] - mx);
+  }
+  __syncthreads();
+  float acc[NE];
+#pragma unroll
+  for (int k = 0; k < NE; ++k) acc[k] = 0.f;
+  for (int f = 0; f < m; ++f) {
+#pragma unroll
+    for (int k = 0; k < NE; ++k) {
+      const int e = tid + k * kThreads;
+      if (e < kQT * D1) {
+        const int r = e / D1, c = e % D1;
+        acc[k] = fmaf(U[r * mp + f], Sh[static_cast<size_t>(f) * D1 + c], acc[k]);
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < NE; ++k) {
+    const int e = tid + k * kThreads;
+    if (e < kQT * D1) O[(e / D1) * (D1 + 1) + e % D1] = acc[k];
+  }
+  __syncthreads();
+  T* Oh = out + static_cast<size_t>(bh) * L * D;
+  for (int i = tid; i < kQT * D; i += kThreads) {
+    const int r = i / D, c = i % D;
+    if (r < qw) store_as(&Oh[static_cast<size_t>(q0 + r) * D + c], O[r * (D1 + 1) + c] / O[r * (D1 + 1) + D]);
+  }
+}
+
+template <typename T, int D>
+int launch_key(const void* K, const void* V, const float* W, void* partials, const Plan& p,
+               cudaStream_t st) {
+  constexpr int D1 = D + 1;
+  const size_t smem = sizeof(float) * (kFB * D1 + 2 * kTT * D1 + kTT * (kFB + 1) + kThreads / 32);
+  auto kern = key_pass_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "key pass attribute: %s", cudaGetErrorString(e));
+  dim3 grid(p.P, p.B * p.Hkv, p.nsb);
+  char* base = static_cast<char*>(partials);
+  kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(K), static_cast<const T*>(V), W,
+                                     reinterpret_cast<float*>(base + p.part_S_off),
+                                     reinterpret_cast<float*>(base + p.part_c_off), p.L, p.m, p.P,
+                                     p.chunk, p.nsb, p.wscale, p.nscale);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "key pass launch: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
+template <typename T, int D>
+int launch_query(const void* Q, const float* W, const void* state, void* out, const Plan& p,
+                 cudaStream_t st) {
+  constexpr int D1 = D + 1;
+  const size_t smem = sizeof(float) * (kQT * D1 + kFB * D1 + kQT * (D1 + 1) + kQT * (p.m + 1));
+  auto kern = query_pass_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "query pass attribute: %s", cudaGetErrorString(e));
+  dim3 grid((p.L + kQT - 1) / kQT, p.B * p.H);
+  const char* base = static_cast<const char*>(state);
+  kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(Q), W,
+                                     reinterpret_cast<const float*>(base + p.st_S_off),
+                                     static_cast<T*>(out), p.L, p.m, p.H, p.Hkv, p.wscale);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "query pass launch: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
+}  // namespace
+
+int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials,
+                  const Plan& p, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FAVOR_F32)
+    return p.d == 64 ? launch_key<float, 64>(K, V, W, partials, p, st) : launch_key<float, 128>(K, V, W, partials, p, st);
+  return p.d == 64 ? launch_key<__nv_bfloat16, 64>(K, V, W, partials, p, st)
+                   : launch_key<__nv_bfloat16, 128>(K, V, W, partials, p, st);
+}
+
+int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int D1 = p.d + 1;
+  dim3 grid((p.m * D1 + kThreads - 1) / kThreads, p.B * p.Hkv);
+  const char* pb = static_cast<const char*>(partials);
+  char* sb = static_cast<char*>(state);
+  state_reduce_kernel<<<grid, kThreads, 0, st>>>(
+      reinterpret_cast<const float*>(pb + p.part_S_off), reinterpret_cast<const float*>(pb + p.part_c_off),
+      reinterpret_cast<float*>(sb + p.st_S_off), reinterpret_cast<float*>(sb + p.st_c_off), p.P, p.m, D1, p.nsb);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "state reduce launch: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
+int simt_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out,
+                    const Plan& p, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FAVOR_F32)
+    return p.d == 64 ? launch_query<float, 64>(Q, W, state, out, p, st) : launch_query<float, 128>(Q, W, state, out, p, st);
+  return p.d == 64 ? launch_query<__nv_bfloat16, 64>(Q, W, state, out, p, st)
+                   : launch_query<__nv_bfloat16, 128>(Q, W, state, out, p, st);
+}
+
+}  // namespace favor

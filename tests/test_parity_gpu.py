@@ -1,0 +1,173 @@
+"""GPU parity: the CUDA path against the fp64 oracle on identical seeded inputs.
+
+Tolerances (fixed for this library): bf16 inputs with fp32 accumulation must
+reach max |gpu - oracle| <= 2e-2 and sum|gpu - oracle| / sum|oracle| <= 5e-3;
+fp32 inputs must reach 1e-4 on both.  The GPU gets W from the library's
+favor_make_features, the oracle from its own generator (the two are checked
+equal on the CPU in test_abi.py).
+"""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+import linear_approximate_softmax_b200 as fv  # noqa: E402
+from linear_approximate_softmax_b200 import workloads as wl  # noqa: E402
+from oracle import favor as ofv  # noqa: E402
+
+TOL = {torch.bfloat16: (2e-2, 5e-3), torch.float32: (1e-4, 1e-4)}
+
+
+def f64(t):
+    return t.float().numpy().astype(np.float64)
+
+
+def gpu_attention(Q, K, V, W):
+    out = fv.favor_attention(Q.cuda(), K.cuda(), V.cuda(), W.cuda())
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+def assert_close(got, ref, dtype, what=""):
+    ma, mr = ofv.error_metrics(f64(got) if torch.is_tensor(got) else got, ref)
+    tol_abs, tol_rel = TOL[dtype]
+    assert np.all(np.isfinite(f64(got) if torch.is_tensor(got) else got)), what
+    assert ma <= tol_abs and mr <= tol_rel, f"{what}: max-abs {ma:.3g} (<= {tol_abs}), mean-rel {mr:.3g} (<= {tol_rel})"
+    return ma, mr
+
+
+def run_case(Q, K, V, m, seed=1, orthogonal=True, what=""):
+    d = Q.shape[-1]
+    W = fv.favor_make_features(seed, m, d, orthogonal)
+    got = gpu_attention(Q, K, V, W)
+    ref = ofv.favor_attention(f64(Q), f64(K), f64(V), ofv.make_features_f32(seed, m, d, orthogonal))
+    return assert_close(got, ref, Q.dtype, what)
+
+
+# ---- the five workloads at sizes the oracle runs element-wise in seconds ----
+SMALL = {
+    "fp32_L256": dict(),
+    "bf16_L4096": dict(B=2, H=2, Hkv=2, L=1000),
+    "bf16_L16384_heavykeys": dict(B=1, H=3, Hkv=3, L=2000),
+    "bf16_mqa_L8192_d128": dict(B=2, H=4, Hkv=1, L=700),
+    "bf16_L131072_m512": dict(B=1, H=2, Hkv=2, L=3000),
+}
+
+
+@pytest.mark.parametrize("name", wl.WORKLOAD_ORDER)
+def test_workload_small_elementwise(name):
+    w = wl.WORKLOADS[name]
+    Q, K, V = wl.make_inputs(w, **SMALL[name])
+    for orth in w.orthogonal:
+        run_case(Q, K, V, w.m, w.w_seed, orth, f"{name} orthogonal={orth}")
+
+
+# ---- edge cases: ragged and tiny L, m not a multiple of 64, grouped heads ----
+@pytest.mark.parametrize("L", [1, 2, 127, 128, 129, 1000])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_ragged_lengths(L, dtype):
+    Q, K, V = wl.random_inputs(1, 2, 1, L, 64, dtype, seed=L)
+    run_case(Q, K, V, 64, what=f"L={L}")
+
+
+@pytest.mark.parametrize("m", [16, 48, 80, 128, 192, 512])
+@pytest.mark.parametrize("d", [64, 128])
+def test_feature_counts(m, d):
+    Q, K, V = wl.random_inputs(1, 2, 2, 300, d, torch.bfloat16, seed=m + d)
+    run_case(Q, K, V, m, what=f"m={m} d={d}")
+
+
+@pytest.mark.parametrize("H,Hkv", [(6, 2), (8, 1), (4, 4)])
+def test_grouped_heads(H, Hkv):
+    Q, K, V = wl.random_inputs(2, H, Hkv, 257, 64, torch.bfloat16, seed=H * 10 + Hkv)
+    run_case(Q, K, V, 128, what=f"H={H} Hkv={Hkv}")
+
+
+def test_large_norm_inputs_stay_finite():
+    # exponents far below zero: only the stabilisers keep exp() in range
+    Q, K, V = wl.random_inputs(1, 1, 1, 500, 64, torch.float32, seed=3, scale=6.0)
+    run_case(Q, K, V, 128, what="scale 6")
+
+
+def test_growing_key_norms_force_rescaling():
+    # key norms rise along the sequence, so later chunks raise the running stabiliser
+    Q, K, V = wl.random_inputs(1, 1, 1, 4000, 64, torch.float32, seed=4)
+    ramp = torch.linspace(0.2, 3.0, 4000).view(1, 1, 4000, 1)
+    run_case(Q, (K * ramp).contiguous(), V, 128, what="ramp")
+
+
+# ---- full sizes, in the launch configuration bench.py times ----------------
+def _full(name, orthogonal=True, heads=2, rows=256):
+    w = wl.WORKLOADS[name]
+    Q, K, V = wl.make_inputs(w)
+    W = fv.favor_make_features(w.w_seed, w.m, w.d, orthogonal)
+    out = gpu_attention(Q, K, V, W)
+    Wo = ofv.make_features_f32(w.w_seed, w.m, w.d, orthogonal)
+    G = w.H // w.Hkv
+    rng = np.random.default_rng(0)
+    got, ref = [], []
+    for bh in rng.choice(w.B * w.H, size=min(heads, w.B * w.H), replace=False):
+        b, h = divmod(int(bh), w.H)
+        S, _ = ofv.key_state(f64(K[b, h // G]), f64(V[b, h // G]), Wo)
+        idx = np.sort(rng.choice(w.L, size=min(rows, w.L), replace=False))
+        idx[-1] = w.L - 1  # always include the ragged end of the sequence
+        ref.append(ofv.query_output(f64(Q[b, h, idx]), Wo, S))
+        got.append(f64(out[b, h, idx]))
+        v = f64(V[b, h // G])
+        o = f64(out[b, h])
+        assert np.all(o >= v.min(0) - 2e-2) and np.all(o <= v.max(0) + 2e-2)  # convex combination
+    assert torch.isfinite(out.float()).all()
+    return assert_close(np.concatenate(got), np.concatenate(ref), w.dtype, f"{name} full")
+
+
+@pytest.mark.parametrize("name", wl.WORKLOAD_ORDER)
+def test_workload_full_size_sampled(name):
+    w = wl.WORKLOADS[name]
+    for orth in w.orthogonal:
+        _full(name, orth)
+
+
+# ---- API equivalences -------------------------------------------------------
+def test_deterministic_bitwise():
+    w = wl.WORKLOADS["bf16_L4096"]
+    Q, K, V = [t.cuda() for t in wl.make_inputs(w, B=2, H=4, Hkv=4, L=4096)]
+    W = fv.favor_make_features(1, w.m, w.d).cuda()
+    a = fv.favor_attention(Q, K, V, W)
+    b = fv.favor_attention(Q, K, V, W)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_stage_calls_equal_fused_call_and_state_matches_oracle(dtype):
+    B, H, Hkv, L, d, m = 2, 4, 2, 1500, 64, 192
+    Q, K, V = wl.random_inputs(B, H, Hkv, L, d, dtype, seed=11)
+    W = fv.favor_make_features(1, m, d)
+    Qd, Kd, Vd, Wd = Q.cuda(), K.cuda(), V.cuda(), W.cuda()
+    part = torch.empty(fv.favor_partials_bytes(B, Hkv, L, d, m), dtype=torch.uint8, device="cuda")
+    state = torch.empty(fv.favor_state_bytes(B, Hkv, d, m), dtype=torch.uint8, device="cuda")
+    fv.favor_key_pass(Kd, Vd, Wd, part)
+    fv.favor_state_reduce(part, state, B, Hkv, L, d, m)
+    out = torch.empty_like(Qd)
+    fv.favor_query_pass(Qd, Wd, state, Hkv, out)
+    fused = fv.favor_attention(Qd, Kd, Vd, Wd)
+    torch.cuda.synchronize()
+    assert torch.equal(out, fused)
+    S, _ = fv.state_views(state, B, Hkv, d, m)
+    Wo = ofv.make_features_f32(1, m, d)
+    for b in range(B):
+        for g in range(Hkv):
+            So, _ = ofv.key_state(f64(K[b, g]), f64(V[b, g]), Wo)
+            Sg = S[b * Hkv + g].double().cpu().numpy()
+            # the state is defined up to one positive constant (stabiliser, 1/sqrt(m))
+            np.testing.assert_allclose(Sg / Sg[:, d].sum(), So / So[:, d].sum(), rtol=1e-3, atol=1e-6)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_host_call_equals_device_call(dtype):
+    Q, K, V = wl.random_inputs(1, 2, 1, 777, 128, dtype, seed=5)
+    W = fv.favor_make_features(1, 128, 128)
+    host = fv.favor_attention_host(Q.pin_memory(), K.pin_memory(), V.pin_memory(), W)
+    dev = gpu_attention(Q, K, V, W)
+    assert torch.equal(host, dev)
