@@ -158,6 +158,33 @@ FAVOR_API int favor_state_reduce(const void* partials, void* state, int B, int H
 FAVOR_API int favor_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out,
                      int B, int H, int Hkv, int L, int d, int m, favor_stream_t stream);
 
+/*
+ * favor_attention_noalloc — favor_attention for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this call; it serves the library's users.
+ * favor_attention allocates its scratch on every call.  A caller whose device
+ * memory is owned and budgeted by its own allocator, or whose serving loop
+ * cannot afford an allocator call, uses this entry point instead: it computes
+ * the same result and allocates nothing, using a 16 MiB array in device
+ * global memory that is part of the library (every GPU that loads the
+ * library's kernels holds it until the process exits).
+ *
+ * dtype: FAVOR_BF16 or FAVOR_F32 for Q, K, V and out; other arguments as for
+ * favor_attention (device pointers, caller-owned, 16-byte aligned).
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * To fit, the key pass may be split into fewer chunks than favor_attention
+ * uses, so results can differ from it in the last bits.  Shapes whose state
+ * alone does not fit return FAVOR_ERR_UNSUPPORTED with the sizes in
+ * favor_last_error().  Every call shares the one array and overwrites all of
+ * the scratch it uses, so nothing has to be cleared between calls, but calls
+ * that overlap on the GPU (on different streams, or from different threads)
+ * race on it: serialise them.
+ */
+FAVOR_API int favor_attention_noalloc(int dtype, const void* Q, const void* K, const void* V, const float* W,
+                                      void* out, int B, int H, int Hkv, int L, int d, int m,
+                                      favor_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

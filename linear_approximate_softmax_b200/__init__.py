@@ -5,7 +5,7 @@ current CUDA stream) into the C ABI declared in include/favor.h; all of the
 arithmetic runs in the library's CUDA kernels.  PyTorch supplies device memory
 and streams.  The names match the C entry points.
 
-The library must have been built (``python -m linear_approximate_softmax_b200.build``);
+The library must have been built (``python linear_approximate_softmax_b200/build.py``);
 importing this package without it raises ImportError — there is no fallback.
 """
 import ctypes
@@ -27,11 +27,11 @@ FAVOR_F32 = 1
 EXPORTS = [
     "favor_last_error", "favor_version", "favor_make_features", "favor_attention",
     "favor_attention_f32", "favor_attention_host", "favor_partials_bytes", "favor_state_bytes",
-    "favor_key_pass", "favor_state_reduce", "favor_query_pass",
+    "favor_key_pass", "favor_state_reduce", "favor_query_pass", "favor_attention_noalloc",
 ]
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m linear_approximate_softmax_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python linear_approximate_softmax_b200/build.py`")
 lib = ctypes.CDLL(LIB_PATH)
 
 _i, _p, _sz, _u64 = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64
@@ -57,6 +57,8 @@ lib.favor_state_reduce.argtypes = [_p, _p, _i, _i, _i, _i, _i, _p]
 lib.favor_state_reduce.restype = _i
 lib.favor_query_pass.argtypes = [_i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
 lib.favor_query_pass.restype = _i
+lib.favor_attention_noalloc.argtypes = [_i] + _ATT
+lib.favor_attention_noalloc.restype = _i
 
 
 class FavorError(RuntimeError):
@@ -141,6 +143,18 @@ def favor_attention_host(Q, K, V, W, out=None, stream=None):
                                     ctypes.c_void_p(V.data_ptr()), ctypes.c_void_p(W.data_ptr()),
                                     ctypes.c_void_p(out.data_ptr()), B, H, Hkv, L, d, m, _stream(stream)),
            "favor_attention_host")
+    return out
+
+
+def favor_attention_noalloc(Q, K, V, W, out=None, stream=None):
+    """favor_attention without any device allocation (scratch in the library's static array)."""
+    code = _dtype_code(Q)
+    B, H, Hkv, L, d, m = _shape(Q, K, V, W)
+    if out is None:
+        out = torch.empty_like(Q)
+    _check(lib.favor_attention_noalloc(code, _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(W, "W"),
+                                       _dev(out, "out"), B, H, Hkv, L, d, m, _stream(stream)),
+           "favor_attention_noalloc")
     return out
 
 

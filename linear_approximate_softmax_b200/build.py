@@ -1,6 +1,6 @@
 """Build libfavor_b200.so in-tree for sm_100a with nvcc.
 
-Usage: python -m linear_approximate_softmax_b200.build  (or call build()).
+Usage: python linear_approximate_softmax_b200/build.py [-f] [-v]  (or call build()).
 Objects go to _build/ at the repository root; the shared library is written
 next to this file so that it travels with the package.
 """
@@ -15,7 +15,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfavor_b200.so")
 
-SOURCES = ["favor_api.cu", "favor_features.cpp", "kernels_simt.cu"]
+SOURCES = ["favor_api.cu", "favor_features.cpp", "kernels_simt.cu", "favor_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC]
 

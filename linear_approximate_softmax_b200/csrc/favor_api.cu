@@ -109,7 +109,18 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
   return FAVOR_OK;
 }
 
-namespace {
+void plan_limit_chunks(Plan* p, int max_P) {
+  if (max_P < 1) max_P = 1;
+  if (p->P <= max_P) return;
+  const int heads = p->B * p->Hkv;
+  const int tiles = (p->L + kTileTokens - 1) / kTileTokens;
+  const int chunk_tiles = (tiles + max_P - 1) / max_P;
+  p->chunk = chunk_tiles * kTileTokens;
+  p->P = (tiles + chunk_tiles - 1) / chunk_tiles;
+  const size_t D1 = static_cast<size_t>(p->d) + 1;
+  p->part_c_off = round_up(sizeof(float) * heads * p->P * p->m * D1, 256);
+  p->part_bytes = p->part_c_off + round_up(sizeof(float) * heads * p->P * p->nsb, 256);
+}
 
 int run_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials, const Plan& p,
                  cudaStream_t st) {
@@ -124,6 +135,8 @@ int run_query_pass(int dtype, const void* Q, const float* W, const void* state, 
                    cudaStream_t st) {
   return simt_query_pass(dtype, Q, W, state, out, p, st);
 }
+
+namespace {
 
 int attention_impl(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,
                    int H, int Hkv, int L, int d, int m, cudaStream_t st) {

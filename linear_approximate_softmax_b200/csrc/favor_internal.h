@@ -6,6 +6,9 @@
 
 #include "favor.h"
 
+struct CUstream_st;
+typedef struct CUstream_st* cudaStream_t;
+
 namespace favor {
 
 // Records `msg` as the calling thread's last error and returns `code`.
@@ -34,6 +37,17 @@ struct Plan {
 
 // Fills `p` for a validated shape on the current device.  Returns FAVOR_OK or an error.
 int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p);
+
+// Re-splits the key pass of `p` into at most max_P chunks per kv head and
+// recomputes the partials layout (the state layout does not depend on it).
+void plan_limit_chunks(Plan* p, int max_P);
+
+// The three steps of the path, each dispatched to its kernel on `st`.
+int run_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials, const Plan& p,
+                 cudaStream_t st);
+int run_reduce(const void* partials, void* state, const Plan& p, cudaStream_t st);
+int run_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out, const Plan& p,
+                   cudaStream_t st);
 
 // ---- CUDA-core kernels (fp32 arithmetic; fp32 or bf16 storage) -------------
 int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials,
