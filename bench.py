@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's B (profiling runs)")
     return ap.parse_args()
 
 
@@ -134,18 +135,22 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
 
 
-def oracle_rate(w, budget_s, max_heads=None):
-    """The fp64 oracle, as it stands, on whole (batch, head) pairs of the workload until the budget is spent."""
-    import numpy as np
+def oracle_rate(w, budget_s, max_heads=None, inputs=None, start=0):
+    """The fp64 oracle, as it stands, on whole (batch, head) pairs of the workload until the budget is spent.
+
+    Input generation and W construction happen before the clock starts; pairs are taken from
+    index `start` on (wrapping), so successive samples cover different heads.
+    """
     from oracle import favor as ofv
     from threadpoolctl import threadpool_info
-    Q, K, V = wl.make_inputs(w)
+    Q, K, V = inputs if inputs is not None else wl.make_inputs(w)
     Wo = ofv.make_features_f32(w.w_seed, w.m, w.d, w.orthogonal[0])
     G = w.H // w.Hkv
     t0 = time.perf_counter()
     heads = 0
     state = {}
-    for bh in range(w.B * w.H):
+    for i in range(w.B * w.H):
+        bh = (start + i) % (w.B * w.H)
         b, h = divmod(bh, w.H)
         key = (b, h // G)
         if key not in state:
@@ -165,17 +170,16 @@ def run_reference(args, rank, world):
         return
     w = wl.WORKLOADS[args.workload]
     steps = args.steps or 3
-    for _ in range(args.warmup and 1):
-        oracle_rate(w, 0.0, max_heads=1)
-    rates = []
-    t0 = time.perf_counter()
-    total_heads = 0
-    for _ in range(steps):
-        r, heads, dt, threads = oracle_rate(w, 1.0, max_heads=2)
-        rates.append(r)
+    inputs = wl.make_inputs(w)
+    for _ in range(min(args.warmup, 1)):
+        oracle_rate(w, 0.0, max_heads=1, inputs=inputs)
+    total_heads, busy = 0, 0.0
+    for k in range(steps):  # each step: one bounded sample of 2 (batch, head) pairs
+        r, heads, dt, threads = oracle_rate(w, 1.0, max_heads=2, inputs=inputs, start=2 * k)
         total_heads += heads
-    wall = time.perf_counter() - t0
-    value = total_heads * w.L / wall / 1e6
+        busy += dt
+    value = total_heads * w.L / busy / 1e6
+    wall = busy
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
         "warmup": args.warmup, "ms_per_step": wall / steps * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -214,6 +218,9 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = wl.WORKLOADS[args.workload]
+    if args.batch:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch, name=f"{w.name}_B{args.batch}")
     Qh, Kh, Vh = wl.make_inputs(w)
     Wh = fv.favor_make_features(w.w_seed, w.m, w.d, w.orthogonal[0])
     Q, K, V, W = Qh.to(dev), Kh.to(dev), Vh.to(dev), Wh.to(dev)

@@ -51,6 +51,7 @@ typedef struct CUstream_st* favor_stream_t; /* the same type as cudaStream_t */
 #define FAVOR_ERR_UNSUPPORTED (-2) /* shape outside the supported set (see above)     */
 #define FAVOR_ERR_CUDA (-3)        /* a CUDA runtime call or launch failed            */
 #define FAVOR_ERR_NOMEM (-4)       /* a host or device allocation failed              */
+#define FAVOR_ERR_TIMEOUT (-5)     /* a GPU kernel gave up waiting (see favor_device_check) */
 
 /* Element type of Q, K, V and out. */
 #define FAVOR_BF16 0
@@ -61,6 +62,16 @@ FAVOR_API const char* favor_last_error(void);
 
 /* Library version, e.g. 100 for 0.1.0. */
 FAVOR_API int favor_version(void);
+
+/*
+ * favor_device_check — synchronise `stream`, then read and clear the library's
+ * device error word.  The tensor-core kernels bound every wait inside their
+ * pipelines; a CTA that gives up (after 2 s) stops, frees its tensor memory and
+ * sets the word, and its outputs are then undefined.  Returns FAVOR_OK,
+ * FAVOR_ERR_TIMEOUT if any kernel gave up since the last check, or
+ * FAVOR_ERR_CUDA.  The word is per device and shared by all streams.
+ */
+FAVOR_API int favor_device_check(favor_stream_t stream);
 
 /*
  * favor_make_features — the random-feature matrix W (host only, no GPU).

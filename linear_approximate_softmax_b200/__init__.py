@@ -21,13 +21,14 @@ FAVOR_ERR_INVALID = -1
 FAVOR_ERR_UNSUPPORTED = -2
 FAVOR_ERR_CUDA = -3
 FAVOR_ERR_NOMEM = -4
+FAVOR_ERR_TIMEOUT = -5
 FAVOR_BF16 = 0
 FAVOR_F32 = 1
 
 EXPORTS = [
     "favor_last_error", "favor_version", "favor_make_features", "favor_attention",
     "favor_attention_f32", "favor_attention_host", "favor_partials_bytes", "favor_state_bytes",
-    "favor_key_pass", "favor_state_reduce", "favor_query_pass", "favor_attention_noalloc",
+    "favor_key_pass", "favor_state_reduce", "favor_query_pass", "favor_attention_noalloc", "favor_device_check",
 ]
 
 if not os.path.exists(LIB_PATH):
@@ -57,6 +58,8 @@ lib.favor_state_reduce.argtypes = [_p, _p, _i, _i, _i, _i, _i, _p]
 lib.favor_state_reduce.restype = _i
 lib.favor_query_pass.argtypes = [_i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
 lib.favor_query_pass.restype = _i
+lib.favor_device_check.argtypes = [_p]
+lib.favor_device_check.restype = _i
 lib.favor_attention_noalloc.argtypes = [_i] + _ATT
 lib.favor_attention_noalloc.restype = _i
 
@@ -103,6 +106,11 @@ def _shape(Q, K, V, W):
 
 def favor_version():
     return lib.favor_version()
+
+
+def favor_device_check(stream=None):
+    """Synchronise the stream and raise FavorError if a GPU kernel gave up waiting."""
+    _check(lib.favor_device_check(_stream(stream)), "favor_device_check")
 
 
 def favor_make_features(seed, m, d, orthogonal=True):

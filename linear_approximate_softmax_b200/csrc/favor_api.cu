@@ -88,13 +88,22 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
   p->B = B; p->H = H; p->Hkv = Hkv; p->L = L; p->d = d; p->m = m;
   const int heads = B * Hkv;
   const int tiles = (L + kTileTokens - 1) / kTileTokens;
-  // About two key-pass CTAs per SM for each 64-feature block of every kv head.
-  long want = (2L * sms + heads - 1) / heads;
-  if (want < 1) want = 1;
-  if (want > tiles) want = tiles;
-  const int chunk_tiles = (tiles + static_cast<int>(want) - 1) / static_cast<int>(want);
-  p->chunk = chunk_tiles * kTileTokens;
-  p->P = (tiles + chunk_tiles - 1) / chunk_tiles;
+  // Key chunks: the tensor-core key pass runs one CTA per SM for each (kv head,
+  // 128-feature group, chunk).  Pick the chunk count that minimises the
+  // makespan in waves of CTAs, counting half a tile of start-up per wave.
+  const long units = static_cast<long>(heads) * ((m + 127) / 128);
+  double best = 1e300;
+  int best_ct = tiles;
+  for (int P = 1; P <= tiles; ++P) {
+    const int ct = (tiles + P - 1) / P;
+    const long Pe = (tiles + ct - 1) / ct;
+    if (Pe != P) continue;
+    const long waves = (units * Pe + sms - 1) / sms;
+    const double cost = static_cast<double>(waves) * (ct + 0.5);
+    if (cost < best - 1e-9) { best = cost; best_ct = ct; }
+  }
+  p->chunk = best_ct * kTileTokens;
+  p->P = (tiles + best_ct - 1) / best_ct;
   p->nsb = (m + kStabBlock - 1) / kStabBlock;
   const size_t D1 = static_cast<size_t>(d) + 1;
   p->part_S_off = 0;
@@ -103,7 +112,10 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
   p->st_S_off = 0;
   p->st_c_off = round_up(sizeof(float) * heads * m * D1, 256);
   p->st_op_off = p->st_c_off + round_up(sizeof(float) * heads, 256);
-  p->st_bytes = p->st_op_off;
+  p->op_rows = d + 16;
+  p->op_atoms = (m + 31) / 32;
+  p->op_bytes = static_cast<size_t>(p->op_rows) * 128 * p->op_atoms;
+  p->st_bytes = p->st_op_off + round_up(p->op_bytes * heads, 256);
   p->wscale = static_cast<float>(std::pow(static_cast<double>(d), -0.25) * kLog2e);
   p->nscale = static_cast<float>(std::pow(static_cast<double>(d), -0.5) * kLog2e * 0.5);
   return FAVOR_OK;
@@ -124,6 +136,7 @@ void plan_limit_chunks(Plan* p, int max_P) {
 
 int run_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials, const Plan& p,
                  cudaStream_t st) {
+  if (dtype == FAVOR_BF16 && sm100_key_supported(p)) return sm100_key_pass(K, V, W, partials, p, st);
   return simt_key_pass(dtype, K, V, W, partials, p, st);
 }
 
@@ -133,10 +146,26 @@ int run_reduce(const void* partials, void* state, const Plan& p, cudaStream_t st
 
 int run_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out, const Plan& p,
                    cudaStream_t st) {
+  if (dtype == FAVOR_BF16 && sm100_query_supported(p)) return sm100_query_pass(Q, W, state, out, p, st);
   return simt_query_pass(dtype, Q, W, state, out, p, st);
 }
 
 namespace {
+
+// Stream-ordered scratch is returned to the device's default pool after each
+// call; by default the pool unmaps it at the next synchronisation, so the
+// next call maps it again.  Keep it mapped (once per device, this process only).
+void keep_pool_mapped() {
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || done[dev]) return;
+  cudaMemPool_t pool;
+  if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+    uint64_t threshold = UINT64_MAX;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &threshold);
+  }
+  done[dev] = true;
+}
 
 int attention_impl(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,
                    int H, int Hkv, int L, int d, int m, cudaStream_t st) {
@@ -144,6 +173,7 @@ int attention_impl(int dtype, const void* Q, const void* K, const void* V, const
   FAVOR_TRY(check_ptrs("favor_attention", {Q, K, V, W, out}));
   Plan p;
   FAVOR_TRY(make_plan(B, H, Hkv, L, d, m, &p));
+  keep_pool_mapped();
   void* ws = nullptr;
   const size_t st_off = round_up(p.part_bytes, 256);
   FAVOR_CUDA_TRY(cudaMallocAsync(&ws, st_off + p.st_bytes, st), "favor_attention scratch allocation");
@@ -192,6 +222,7 @@ int favor_attention_host(int dtype, const void* Q, const void* K, const void* V,
   const size_t nq = static_cast<size_t>(B) * H * L * d, nk = static_cast<size_t>(B) * Hkv * L * d;
   const size_t bq = round_up(nq * es, 256), bk = round_up(nk * es, 256), bw = round_up(sizeof(float) * m * d, 256);
   void* buf = nullptr;
+  keep_pool_mapped();
   FAVOR_CUDA_TRY(cudaMallocAsync(&buf, 2 * bq + 2 * bk + bw, st), "favor_attention_host device allocation");
   char* dQ = static_cast<char*>(buf);
   char* dK = dQ + bq;
@@ -215,6 +246,15 @@ int favor_attention_host(int dtype, const void* Q, const void* K, const void* V,
   if (rc != FAVOR_OK) return rc;
   if (fe != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "favor_attention_host release: %s", cudaGetErrorString(fe));
   if (se != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "favor_attention_host: %s", cudaGetErrorString(se));
+  return FAVOR_OK;
+}
+
+int favor_device_check(favor_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "favor_device_check: %s", cudaGetErrorString(e));
+  unsigned int word = 0;
+  FAVOR_TRY(sm100_read_and_clear_error(&word));
+  if (word) return set_errorf(FAVOR_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (error word 0x%x)", word);
   return FAVOR_OK;
 }
 

@@ -31,6 +31,12 @@ struct Plan {
   size_t part_S_off, part_c_off, part_bytes;
   // byte offsets inside the state buffer
   size_t st_S_off, st_c_off, st_op_off, st_bytes;
+  // The state re-packed as the fp32 (tf32) B operand of the query pass's
+  // second MMA: per kv head, op_atoms blocks of 32 features, each op_rows rows
+  // (output column n: d value columns, the normaliser at n = d, zeros after) of
+  // 128 B, K-major with the 128-byte swizzle (16-byte chunk c of row n at c ^ (n % 8)).
+  int op_rows, op_atoms;
+  size_t op_bytes;
   float wscale;     // d^-1/4 * log2(e): W is multiplied by this on the device
   float nscale;     // d^-1/2 * log2(e) / 2: |k|^2 is multiplied by this
 };
@@ -55,5 +61,13 @@ int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void*
 int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream);
 int simt_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out,
                     const Plan& p, void* stream);
+
+// ---- tensor-core kernels (sm_100a, bf16 storage) ------------------------------
+bool sm100_key_supported(const Plan& p);
+bool sm100_query_supported(const Plan& p);
+int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st);
+int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st);
+// Reads and clears the device error word (bit 0: a bounded wait gave up).
+int sm100_read_and_clear_error(unsigned int* word);
 
 }  // namespace favor

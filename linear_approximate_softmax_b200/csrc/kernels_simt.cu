@@ -149,26 +149,40 @@ __global__ void __launch_bounds__(kThreads) key_pass_kernel(
   if (tid == 0) part_c[(static_cast<size_t>(head) * P + p) * nsb + fb] = c_run;
 }
 
-// grid (ceil(m*(d+1)/256), B*Hkv), 256 threads.  Fixed summation order p = 0..P-1.
+// grid (ceil(op_atoms*32*op_rows/256), B*Hkv), 256 threads.  One thread per
+// (feature f, column n) of the padded state: it sums the chunk partials in the
+// fixed order p = 0..P-1, each rescaled from its chunk stabiliser to the
+// largest one, writes S[f][n] (fp32) and the fp32 operand image of the query
+// pass (zeros in the padding).
 __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
     const float* __restrict__ part_S, const float* __restrict__ part_c, float* __restrict__ S,
-    float* __restrict__ Sc, int P, int m, int D1, int nsb) {
+    float* __restrict__ Sc, unsigned char* __restrict__ op, int P, int m, int D1, int nsb, int op_rows,
+    int op_atoms, size_t op_bytes) {
   const int head = blockIdx.y;
   const int e = blockIdx.x * kThreads + threadIdx.x;
   const float* pc = part_c + static_cast<size_t>(head) * P * nsb;
   float cs = -INFINITY;
   for (int i = 0; i < P * nsb; ++i) cs = fmaxf(cs, pc[i]);
-  if (e < m * D1) {
-    const int sb = (e / D1) / kStabBlock;
-    float s = 0.f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) Sc[head] = cs;
+  if (e >= op_atoms * 32 * op_rows) return;
+  const int f = e / op_rows, n = e % op_rows;
+  float val = 0.f;
+  if (f < m && n < D1) {
+    const int sb = f / kStabBlock;
+    const size_t idx = static_cast<size_t>(f) * D1 + n;
+    float acc = 0.f;
     for (int p = 0; p < P; ++p) {
       const float c = pc[p * nsb + sb];
       const float w = (c == -INFINITY) ? 0.f : exp2f(c - cs);
-      s = fmaf(w, part_S[(static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * D1 + e], s);
+      acc = fmaf(w, part_S[(static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * D1 + idx], acc);
     }
-    S[static_cast<size_t>(head) * m * D1 + e] = s;
+    S[static_cast<size_t>(head) * m * D1 + idx] = acc;
+    val = acc;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) Sc[head] = cs;
+  const int atom = f >> 5, chunk = (f & 31) >> 2, el = f & 3;
+  const size_t off = static_cast<size_t>(atom) * op_rows * 128 + static_cast<size_t>(n) * 128 +
+                     ((chunk ^ (n & 7)) << 4) + el * 4;
+  *reinterpret_cast<float*>(op + static_cast<size_t>(head) * op_bytes + off) = val;
 }
 
 // grid (ceil(L/32), B*H), 256 threads.
@@ -301,12 +315,13 @@ int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void*
 int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int D1 = p.d + 1;
-  dim3 grid((p.m * D1 + kThreads - 1) / kThreads, p.B * p.Hkv);
+  dim3 grid((p.op_atoms * 32 * p.op_rows + kThreads - 1) / kThreads, p.B * p.Hkv);
   const char* pb = static_cast<const char*>(partials);
   char* sb = static_cast<char*>(state);
   state_reduce_kernel<<<grid, kThreads, 0, st>>>(
       reinterpret_cast<const float*>(pb + p.part_S_off), reinterpret_cast<const float*>(pb + p.part_c_off),
-      reinterpret_cast<float*>(sb + p.st_S_off), reinterpret_cast<float*>(sb + p.st_c_off), p.P, p.m, D1, p.nsb);
+      reinterpret_cast<float*>(sb + p.st_S_off), reinterpret_cast<float*>(sb + p.st_c_off),
+      reinterpret_cast<unsigned char*>(sb + p.st_op_off), p.P, p.m, D1, p.nsb, p.op_rows, p.op_atoms, p.op_bytes);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "state reduce launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;

@@ -1,0 +1,823 @@
+// FAVOR+ on the sm_100a tensor cores (tcgen05 + TMEM + TMA), bf16 inputs.
+//
+// "Rethinking Attention with Performers" (Abstract; 제안 방법 / proposed
+// method): out = phi(Q')(phi(K')^T [V|1]) / last column, with positive random
+// features phi(x') = exp(W x' - |x'|^2/2)/sqrt(m).  Both contractions on each
+// side are dense, so they run on the tensor cores; the exp feature map (m
+// exponentials per token) runs on the MUFU between them.
+//
+// Key pass (one CTA per 128-feature group x key chunk x kv head), transposed:
+//   MMA1  U^T[f, t] = W'[f, :] . K[t, :]      A = W' (hi + lo bf16) in TMEM,  B = K tile (TMA, smem)
+//   exp   phi^T[f, t] = 2^(U^T - n(k_t) - c)  written back over U^T as bf16 (A operand of MMA2)
+//   MMA2  S[f, :] += phi^T[f, :] . [V | 1]    A = phi^T in TMEM, B = V tile (smem, MN-major) and a ones tile
+// so every thread of the two epilogue warpgroups owns one feature (TMEM lane)
+// and half of the tile's tokens.  c is the chunk's running max exponent, raised
+// only when a tile exceeds it by more than 2^8 (the accumulator is then rescaled
+// exactly); the state reduction later brings all chunks to one constant.
+//
+// Query pass (one CTA per SM over a contiguous range of 128-query tiles):
+//   MMA1  U[q, f] = Q[q, :] . W'[f, :]        A = Q tile (TMA), B = W' hi + lo (smem), per 128-feature block
+//   exp   phi[q, f] = 2^(U - c_q)             fp32, written back over U; c_q = the row max,
+//                                             raised lazily across feature blocks
+//   MMA2  O[q, :] += phi[q, block] . S'[block, :]   kind::tf32: A = phi in TMEM, B = fp32 state image (smem)
+//   out = O[:, :d] / O[:, d] -> bf16 -> TMA store.
+// MMA2 runs in tf32 rather than bf16 because rounding the state to bf16 costs up to
+// 2^-8 of an output when one feature dominates a query, which, with the bf16 output
+// rounding on top, reaches the 2e-2 max-abs bound.
+//
+// W' = d^-1/4 log2(e) W is split as W' = hi + lo in bf16 so that the exponent
+// arguments keep ~17 bits: a single bf16 W' moves the exponents by up to
+// 2^-9 |W'x|, which fails the bf16 output tolerance on heavy-tailed keys.
+//
+// Every mbarrier wait is bounded (2 s); a CTA that gives up raises the device
+// error word, stops issuing work, drains its own copies and frees its TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "favor_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace favor {
+
+__device__ unsigned int g_sm100_error_word;
+
+namespace {
+using namespace sm100;
+
+constexpr int kThreads = 384;  // 12 warps: producer, MMA, two spare/norm warps, 8 epilogue warps
+constexpr int kEpiWarp0 = 4;
+constexpr int kEpiThreads = 256;
+constexpr uint32_t kBarEpi = 1;    // named barrier: epilogue max exchange
+constexpr uint32_t kBarStore = 2;  // named barrier: output staging
+constexpr float kTau = 8.f;        // lazy stabiliser threshold (log2 units)
+
+__device__ __forceinline__ uint32_t taddr(uint32_t base, int lane_quarter, int col) {
+  return base + (static_cast<uint32_t>(lane_quarter * 32) << 16) + static_cast<uint32_t>(col);
+}
+
+// ============================================================================
+// Key pass
+// ============================================================================
+template <int D>
+struct KeyCfg {
+  static constexpr int NST = (D == 64) ? 4 : 2;   // K/V pipeline stages
+  static constexpr int NB1 = (D == 64) ? 2 : 1;   // U^T buffers in TMEM
+  static constexpr int RGN = 128 * 64 * 2;        // one 128-token x 64-dim swizzled region
+  static constexpr int TILE = RGN * (D / 64);     // one K (or V) tile
+  static constexpr int NS = D + 16;               // S columns: D values, then the ones block
+  // TMEM columns
+  static constexpr int T_WHI = 0;
+  static constexpr int T_WLO = D / 2;
+  static constexpr int T_D1 = D;
+  static constexpr int T_S = D + NB1 * 128;
+  static_assert(T_S + NS <= 512, "TMEM budget");
+  // shared memory, from a 1024-aligned base
+  static constexpr int S_K = 0;
+  static constexpr int S_V = S_K + NST * TILE;
+  static constexpr int S_ONES = S_V + NST * TILE;  // 2 atoms x 16 rows x 128 B
+  static constexpr int S_NRM = S_ONES + 4096;      // NST x 128 floats
+  static constexpr int S_RED = S_NRM + NST * 512;  // 2 x 8 floats
+  static constexpr int S_BAR = S_RED + 64;
+  // barriers: kv_full[NST], kv_empty[NST], nrm_ready[NST], d1_full[NB1], phi_ready[NB1], s_done
+  static constexpr int B_KVF = 0, B_KVE = NST, B_NRM = 2 * NST, B_D1F = 3 * NST, B_PHI = 3 * NST + NB1,
+                       B_SDONE = 3 * NST + 2 * NB1, NBAR = 3 * NST + 2 * NB1 + 1;
+  static constexpr int S_TPTR = S_BAR + NBAR * 8;
+  static constexpr int S_ABORT = S_TPTR + 8;
+  static constexpr int SMEM = S_ABORT + 16 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const float* __restrict__ W,
+    float* __restrict__ part_S, float* __restrict__ part_c, int L, int m, int P, int chunk, int nsb, float wscale,
+    float nscale) {
+  using C = KeyCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the feature groups of one (kv head, chunk) are adjacent CTAs, so they run together and the
+  // second group's K/V reads hit L2
+  const int grp = blockIdx.x, p = blockIdx.y, head = blockIdx.z;
+  const int f0 = grp * 128, gw = min(128, m - f0);
+  const int t_begin = p * chunk, t_end = min(L, t_begin + chunk);
+  const int ntiles = (t_end - t_begin + 127) / 128;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
+  uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
+  float* nrm = reinterpret_cast<float*>(smem + C::S_NRM);
+  float* red = reinterpret_cast<float*>(smem + C::S_RED);
+  auto bar = [&](int i) { return sbase + C::S_BAR + 8u * i; };
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(bar(C::B_KVF + s), 1);
+      mbar_init(bar(C::B_KVE + s), 1);
+      mbar_init(bar(C::B_NRM + s), 2);
+    }
+    for (int b = 0; b < C::NB1; ++b) {
+      mbar_init(bar(C::B_D1F + b), 1);
+      mbar_init(bar(C::B_PHI + b), kEpiThreads / 32);
+    }
+    mbar_init(bar(C::B_SDONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tptr_slot), 512);
+    tmem_relinquish();
+  }
+  // ones tile: K-major [16 rows x 128 tokens] in two 64-token atoms; row 0 = 1.0, rows 1..15 = 0
+  for (int i = tid; i < 4096 / 4; i += kThreads) {
+    const int row = (i * 4 % 2048) / 128;
+    reinterpret_cast<uint32_t*>(smem + C::S_ONES)[i] = (row == 0) ? 0x3F803F80u : 0u;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tptr_slot;
+
+  const bool epi = warp >= kEpiWarp0;
+  const int eq = warp & 3;                   // TMEM lane quarter of this warp
+  const int ewg = (warp - kEpiWarp0) >> 2;   // epilogue warpgroup: 0 or 1
+  const int frow = eq * 32 + lane;           // feature row (TMEM lane) owned by an epilogue thread
+  const bool fvalid = frow < gw;
+
+  if (epi) {  // W' = hi + lo (bf16) into TMEM as the A operand of MMA1: lane = feature, 2 dims per column
+    const int f = f0 + frow;
+    uint32_t words[32];
+#pragma unroll
+    for (int half = 0; half < D / 64; ++half) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float w0 = 0.f, w1 = 0.f;
+        if (fvalid) {
+          const float2 v = *reinterpret_cast<const float2*>(W + static_cast<size_t>(f) * D + half * 64 + 2 * j);
+          w0 = v.x * wscale;
+          w1 = v.y * wscale;
+        }
+        if (ewg == 0) {
+          words[j] = pack_bf16x2(w0, w1);
+        } else {
+          const float h0 = __bfloat162float(__float2bfloat16_rn(w0));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(w1));
+          words[j] = pack_bf16x2(w0 - h0, w1 - h1);
+        }
+      }
+      tmem_st32(taddr(tbase, eq, (ewg == 0 ? C::T_WHI : C::T_WLO) + half * 32), words);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  unsigned int* err = &g_sm100_error_word;
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % C::NST;
+        if (i >= C::NST && !mbar_wait(bar(C::B_KVE + s), ((i / C::NST) - 1) & 1, abort_flag, err)) break;
+        mbar_arrive_expect_tx(bar(C::B_KVF + s), 2 * C::TILE);
+        const int t0 = t_begin + 128 * i;
+#pragma unroll
+        for (int r = 0; r < D / 64; ++r) {
+          tma_load_3d(sbase + C::S_K + s * C::TILE + r * C::RGN, &tmK, bar(C::B_KVF + s), 64 * r, t0, head);
+          tma_load_3d(sbase + C::S_V + s * C::TILE + r * C::RGN, &tmV, bar(C::B_KVF + s), 64 * r, t0, head);
+        }
+        issued = i + 1;
+      }
+      // drain: every load this CTA issued must have landed before it exits
+      for (int i = max(0, issued - C::NST); i < issued; ++i)
+        mbar_wait(bar(C::B_KVF + i % C::NST), (i / C::NST) & 1, abort_flag, err, 200000000ull);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t id1 = idesc_bf16(128, 128, false, false);
+      const uint32_t idv = idesc_bf16(128, D, false, true);
+      const uint32_t ido = idesc_bf16(128, 16, false, false);
+      bool ok = true;
+      auto mma2 = [&](int j) {
+        const int s = j % C::NST, b = j % C::NB1;
+        if (!mbar_wait(bar(C::B_PHI + b), (j / C::NB1) & 1, abort_flag, err)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t a = tbase + C::T_D1 + 128 * b + 8 * ks;
+          const uint64_t bv = sdesc_sw128(sbase + C::S_V + s * C::TILE + 2048 * ks, C::RGN, 1024);
+          const uint64_t bo = sdesc_sw128(sbase + C::S_ONES + (ks >> 2) * 2048 + 32 * (ks & 3), 16, 1024);
+          const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
+          mma_ts(tbase + C::T_S, a, bv, idv, acc);
+          mma_ts(tbase + C::T_S + D, a, bo, ido, acc);
+        }
+        mma_commit(bar(C::B_KVE + s));
+        mma_commit(bar(C::B_SDONE));
+        return true;
+      };
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int s = i % C::NST, b = i % C::NB1;
+        if (!mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err)) break;
+        if (i >= C::NB1 && !mbar_wait(bar(C::B_SDONE), (i - C::NB1) & 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t d1 = tbase + C::T_D1 + 128 * b;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t bk = sdesc_sw128(sbase + C::S_K + s * C::TILE + (ks >> 2) * C::RGN + 32 * (ks & 3), 16, 1024);
+          mma_ts(d1, tbase + C::T_WHI + 8 * ks, bk, id1, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t bk = sdesc_sw128(sbase + C::S_K + s * C::TILE + (ks >> 2) * C::RGN + 32 * (ks & 3), 16, 1024);
+          mma_ts(d1, tbase + C::T_WLO + 8 * ks, bk, id1, 1u);
+        }
+        mma_commit(bar(C::B_D1F + b));
+        if (C::NB1 == 2 && i >= 1) ok = mma2(i - 1);
+        if (C::NB1 == 1) ok = mma2(i);
+      }
+      if (ok && C::NB1 == 2 && ntiles >= 1 && !*abort_flag) mma2(ntiles - 1);
+      // all MMAs of this CTA complete before TMEM is released
+      mbar_wait(bar(C::B_SDONE), (ntiles - 1) & 1, abort_flag, err, 200000000ull);
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ---------------- key norms: n(k) = |k|^2 * nscale, +inf past the chunk end ----------------
+    // two warps, two tokens per lane each; the 16-byte chunks of a swizzled row are summed in
+    // any order, and four accumulators keep the FMA chains short
+    const int wsel = warp - 2;
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % C::NST;
+      if (!mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err)) break;
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const int t = lane + 32 * (2 * qq + wsel);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < D / 64; ++r) {
+          const uint4* row = reinterpret_cast<const uint4*>(smem + C::S_K + s * C::TILE + r * C::RGN + t * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = row[c];
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float lo = __uint_as_float(wv[k] << 16), hi = __uint_as_float(wv[k] & 0xFFFF0000u);
+              acc[k] = fmaf(lo, lo, acc[k]);
+              acc[k] = fmaf(hi, hi, acc[k]);
+            }
+          }
+        }
+        const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        nrm[s * 128 + t] = (t_begin + 128 * i + t < t_end) ? sum * nscale : INFINITY;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_NRM + s));
+    }
+  } else if (epi) {
+    // ---------------- epilogue: exp feature map, stabiliser, state readout ----------------
+    float c_run = -INFINITY;
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % C::NST, b = i % C::NB1;
+      mbar_wait(bar(C::B_D1F + b), (i / C::NB1) & 1, abort_flag, err);
+      mbar_wait(bar(C::B_NRM + s), (i / C::NST) & 1, abort_flag, err);
+      tc_fence_after();
+      uint32_t u[64];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(taddr(tbase, eq, C::T_D1 + 128 * b + 64 * ewg), r0);
+        tmem_ld32(taddr(tbase, eq, C::T_D1 + 128 * b + 64 * ewg + 32), r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          u[k] = r0[k];
+          u[32 + k] = r1[k];
+        }
+      }
+      const float4* nv = reinterpret_cast<const float4*>(nrm + s * 128 + 64 * ewg);
+      float a[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k4 = 0; k4 < 16; ++k4) {
+        const float4 n4 = nv[k4];
+        a[4 * k4 + 0] = __uint_as_float(u[4 * k4 + 0]) - n4.x;
+        a[4 * k4 + 1] = __uint_as_float(u[4 * k4 + 1]) - n4.y;
+        a[4 * k4 + 2] = __uint_as_float(u[4 * k4 + 2]) - n4.z;
+        a[4 * k4 + 3] = __uint_as_float(u[4 * k4 + 3]) - n4.w;
+      }
+      if (fvalid) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k) mx = fmaxf(mx, a[k]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) red[(i & 1) * 8 + (warp - kEpiWarp0)] = mx;
+      named_bar_sync(kBarEpi, kEpiThreads);
+      float M = red[(i & 1) * 8];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) M = fmaxf(M, red[(i & 1) * 8 + w]);
+      if (c_run == -INFINITY) {
+        c_run = M;
+      } else if (M > c_run + kTau) {  // uniform across the CTA: rescale S to the new stabiliser
+        mbar_wait(bar(C::B_SDONE), (i - 1) & 1, abort_flag, err);
+        tc_fence_after();
+        const float sc = ex2(c_run - M);
+#pragma unroll
+        for (int cc = 0; cc < C::NS / 16; ++cc) {
+          const int col = C::T_S + ewg * (C::NS / 2) + 8 * cc;
+          uint32_t v[8];
+          tmem_ld8(taddr(tbase, eq, col), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * sc);
+          tmem_st8(taddr(tbase, eq, col), v);
+        }
+        tmem_wait_st();
+        c_run = M;
+      }
+      uint32_t wph[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float p0 = fvalid ? ex2(a[2 * j] - c_run) : 0.f;
+        const float p1 = fvalid ? ex2(a[2 * j + 1] - c_run) : 0.f;
+        wph[j] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(taddr(tbase, eq, C::T_D1 + 128 * b + 32 * ewg), wph);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_PHI + b));
+    }
+    // state readout: S rows of this group -> partial [m][D+1]
+    mbar_wait(bar(C::B_SDONE), (ntiles - 1) & 1, abort_flag, err);
+    tc_fence_after();
+    float* outp = part_S + (static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * (D + 1);
+#pragma unroll
+    for (int cc = 0; cc < C::NS / 16; ++cc) {
+      const int col0 = ewg * (C::NS / 2) + 8 * cc;
+      uint32_t v[8];
+      tmem_ld8(taddr(tbase, eq, C::T_S + col0), v);
+      tmem_wait_ld();
+      if (fvalid) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (col0 + k <= D) outp[static_cast<size_t>(f0 + frow) * (D + 1) + col0 + k] = __uint_as_float(v[k]);
+      }
+    }
+    if (warp == kEpiWarp0 && lane == 0) {
+      for (int sb = 2 * grp; sb < min(nsb, 2 * grp + 2); ++sb)
+        part_c[(static_cast<size_t>(head) * P + p) * nsb + sb] = c_run;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ============================================================================
+// Query pass
+// ============================================================================
+template <int D>
+struct QueryCfg {
+  static constexpr int NSTQ = 2;
+  static constexpr int QTILE = 128 * D * 2;
+  static constexpr int NR = D + 16;                  // output columns of MMA2 (values, normaliser, zeros)
+  static constexpr int MMAX = 256;                   // features held in shared memory
+  static constexpr int SP = NR * 128 * (MMAX / 32);  // the fp32 state image (one buffer)
+  // TMEM columns
+  static constexpr int T_U = 0;        // 2 slots x 128
+  static constexpr int T_O = 256;      // 2 buffers x NR
+  static_assert(T_O + 2 * NR <= 512, "TMEM budget");
+  // shared memory
+  static constexpr int S_WHI = 0;
+  static constexpr int S_WLO = S_WHI + MMAX * 128 * (D / 64);
+  static constexpr int S_SP = S_WLO + MMAX * 128 * (D / 64);
+  static constexpr int S_Q = S_SP + SP;
+  static constexpr int S_OUT = S_Q + NSTQ * QTILE;
+  static constexpr int S_RMX = S_OUT + 2 * QTILE;   // 2 x 2 x 128 floats
+  static constexpr int S_BAR = S_RMX + 2048;
+  // barriers
+  static constexpr int B_QF = 0, B_QE = 2, B_SF = 4, B_SE = 6, B_UF = 8, B_PHI = 10, B_SLOT = 12, B_OF = 14,
+                       B_OE = 16, NBAR = 18;
+  static constexpr int S_TPTR = S_BAR + NBAR * 8;
+  static constexpr int S_ABORT = S_TPTR + 8;
+  static constexpr int SMEM = S_ABORT + 16 + 1024;
+};
+
+struct QueryRange {
+  int T0, T1;  // tiles [T0, T1) of this CTA
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) query_pass_sm100(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, const float* __restrict__ W,
+    const unsigned char* __restrict__ op_img, int L, int m, int H, int Hkv, int ntiles_total, int op_bytes,
+    float wscale) {
+  using C = QueryCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ntq = (L + 127) / 128;
+  const int G = H / Hkv;
+  const int nb = (m + 127) / 128;
+  // contiguous, balanced range of tiles for this CTA
+  const int per = ntiles_total / gridDim.x, extra = ntiles_total % gridDim.x;
+  const int T0 = blockIdx.x * per + min(static_cast<int>(blockIdx.x), extra);
+  const int n = per + (static_cast<int>(blockIdx.x) < extra ? 1 : 0);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
+  uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
+  float* rmx = reinterpret_cast<float*>(smem + C::S_RMX);
+  auto bar = [&](int i) { return sbase + C::S_BAR + 8u * i; };
+  auto kvh_of = [&](int T) {
+    const int bh = T / ntq;
+    return (bh / H) * Hkv + (bh % H) / G;
+  };
+
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::B_QF + i), 1);
+      mbar_init(bar(C::B_QE + i), 1);
+      mbar_init(bar(C::B_SF + i), 1);
+      mbar_init(bar(C::B_SE + i), 1);
+      mbar_init(bar(C::B_UF + i), 1);
+      mbar_init(bar(C::B_PHI + i), kEpiThreads / 32);
+      mbar_init(bar(C::B_SLOT + i), 1);
+      mbar_init(bar(C::B_OF + i), 1);
+      mbar_init(bar(C::B_OE + i), kEpiThreads / 32);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmO);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tptr_slot), 512);
+    tmem_relinquish();
+  }
+  // W' = hi + lo as the K-major, 128B-swizzled B operand of MMA1: row f, 16-byte chunk c at c ^ (f % 8)
+  {
+    const int rows = nb * 128;
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+    for (int item = tid; item < rows * CPR; item += kThreads) {
+      const int f = item / CPR, c = item % CPR;
+      const int rg = c >> 3, cc = c & 7;  // 64-dim region, chunk within the 128-byte row
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float w0 = 0.f, w1 = 0.f;
+        if (f < m) {
+          const float2 v = *reinterpret_cast<const float2*>(W + static_cast<size_t>(f) * D + 8 * c + 2 * k);
+          w0 = v.x * wscale;
+          w1 = v.y * wscale;
+        }
+        hi[k] = pack_bf16x2(w0, w1);
+        const float h0 = __uint_as_float(hi[k] << 16), h1 = __uint_as_float(hi[k] & 0xFFFF0000u);
+        lo[k] = pack_bf16x2(w0 - h0, w1 - h1);
+      }
+      const int off = rg * (C::MMAX * 128) + f * 128 + ((cc ^ (f & 7)) << 4);
+      *reinterpret_cast<uint4*>(smem + C::S_WHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(smem + C::S_WLO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tptr_slot;
+  unsigned int* err = &g_sm100_error_word;
+
+  if (warp == 0) {
+    // ---------------- producer: state images and Q tiles ----------------
+    if (lane == 0) {
+      int k = -1, prev = -1, issued = 0;
+      for (int it = 0; it < n; ++it) {
+        const int T = T0 + it;
+        // the Q tile first: the MMA warp issues the previous head's last MMA2 (which releases
+        // the state image) only after this tile's first MMA1
+        const int s = it % C::NSTQ;
+        if (it >= C::NSTQ && !mbar_wait(bar(C::B_QE + s), ((it / C::NSTQ) - 1) & 1, abort_flag, err)) break;
+        mbar_arrive_expect_tx(bar(C::B_QF + s), C::QTILE);
+        const int bh = T / ntq, qt = T % ntq;
+#pragma unroll
+        for (int r = 0; r < D / 64; ++r)
+          tma_load_3d(sbase + C::S_Q + s * C::QTILE + r * (128 * 128), &tmQ, bar(C::B_QF + s), 64 * r, qt * 128, bh);
+        issued = it + 1;
+        const int kvh = kvh_of(T);
+        if (kvh != prev) {  // new kv head: its state image replaces the previous one once that is released
+          ++k;
+          prev = kvh;
+          if (k >= 1 && !mbar_wait(bar(C::B_SE), (k - 1) & 1, abort_flag, err)) break;
+          mbar_arrive_expect_tx(bar(C::B_SF), op_bytes);
+          bulk_load(sbase + C::S_SP, op_img + static_cast<size_t>(kvh) * op_bytes, op_bytes, bar(C::B_SF));
+        }
+      }
+      for (int it = max(0, issued - C::NSTQ); it < issued; ++it)
+        mbar_wait(bar(C::B_QF + it % C::NSTQ), (it / C::NSTQ) & 1, abort_flag, err, 200000000ull);
+      if (k >= 0) mbar_wait(bar(C::B_SF), k & 1, abort_flag, err, 200000000ull);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t id2 = idesc_tf32(128, C::NR, false, false);
+      int k = -1, prev = -1;  // state image index of the tile whose MMA2s are being issued
+      auto mma2 = [&](int h) {
+        const int it = h / nb, j = h % nb, slot = h & 1, ob = it & 1;
+        if (!mbar_wait(bar(C::B_PHI + slot), (h >> 1) & 1, abort_flag, err)) return false;
+        if (j == 0) {
+          if (it >= 2 && !mbar_wait(bar(C::B_OE + ob), ((it >> 1) - 1) & 1, abort_flag, err)) return false;
+          const int kvh = kvh_of(T0 + it);
+          if (kvh != prev) {
+            ++k;
+            prev = kvh;
+            if (!mbar_wait(bar(C::B_SF), k & 1, abort_flag, err)) return false;
+          }
+        }
+        tc_fence_after();
+        const int bw = min(128, m - 128 * j);
+        for (int ks = 0; ks < bw / 8; ++ks) {  // tf32: 8 features per step, one TMEM column each
+          const int fk = 128 * j + 8 * ks;
+          const uint64_t bd = sdesc_sw128(sbase + C::S_SP + (fk >> 5) * (C::NR * 128) + 32 * ((fk & 31) >> 3), 16, 1024);
+          mma_ts_tf32(tbase + C::T_O + ob * C::NR, tbase + C::T_U + 128 * slot + 8 * ks, bd, id2,
+                      (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(C::B_SLOT + slot));
+        if (j == nb - 1) {
+          mma_commit(bar(C::B_OF + ob));
+          if (it == n - 1 || kvh_of(T0 + it + 1) != prev) mma_commit(bar(C::B_SE));
+        }
+        return true;
+      };
+      bool ok = true;
+      int g = 0;
+      for (int it = 0; it < n && ok; ++it) {
+        const int s = it % C::NSTQ;
+        for (int j = 0; j < nb && ok; ++j, ++g) {
+          const int slot = g & 1;
+          if (j == 0 && !mbar_wait(bar(C::B_QF + s), (it / C::NSTQ) & 1, abort_flag, err)) { ok = false; break; }
+          if (g >= 2 && !mbar_wait(bar(C::B_SLOT + slot), ((g >> 1) - 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const int bw = min(128, m - 128 * j);
+          const uint32_t id1 = idesc_bf16(128, bw, false, false);
+          const uint32_t dU = tbase + C::T_U + 128 * slot;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
+            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * j) * 128 + 32 * (ks & 3);
+            mma_ss(dU, sdesc_sw128(sbase + C::S_Q + s * C::QTILE + qo, 16, 1024),
+                   sdesc_sw128(sbase + C::S_WHI + wo, 16, 1024), id1, ks > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
+            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * j) * 128 + 32 * (ks & 3);
+            mma_ss(dU, sdesc_sw128(sbase + C::S_Q + s * C::QTILE + qo, 16, 1024),
+                   sdesc_sw128(sbase + C::S_WLO + wo, 16, 1024), id1, 1u);
+          }
+          mma_commit(bar(C::B_UF + slot));
+          if (j == nb - 1) mma_commit(bar(C::B_QE + s));
+          if (g >= 1) ok = mma2(g - 1);
+        }
+      }
+      if (ok && g >= 1 && !*abort_flag) mma2(g - 1);
+      if (g >= 1) mbar_wait(bar(C::B_SLOT + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, err, 200000000ull);
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ---------------- epilogue ----------------
+    const int eq = warp & 3, ewg = (warp - kEpiWarp0) >> 2;
+    const int r = eq * 32 + lane;  // query row within the tile (TMEM lane)
+    const bool issuer = (warp == kEpiWarp0 && lane == 0);
+    int g = 0;
+    for (int it = 0; it < n; ++it) {
+      const int ob = it & 1;
+      float c = -INFINITY;
+      for (int j = 0; j < nb; ++j, ++g) {
+        const int slot = g & 1;
+        mbar_wait(bar(C::B_UF + slot), (g >> 1) & 1, abort_flag, err);
+        tc_fence_after();
+        float u[64];
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(taddr(tbase, eq, C::T_U + 128 * slot + 64 * ewg), r0);
+          tmem_ld32(taddr(tbase, eq, C::T_U + 128 * slot + 64 * ewg + 32), r1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            u[k] = __uint_as_float(r0[k]);
+            u[32 + k] = __uint_as_float(r1[k]);
+          }
+        }
+        const int fb = 128 * j + 64 * ewg;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          if (fb + k >= m) u[k] = -INFINITY;
+          mx = fmaxf(mx, u[k]);
+        }
+        rmx[(g & 1) * 256 + ewg * 128 + r] = mx;
+        named_bar_sync(kBarEpi, kEpiThreads);
+        const float M = fmaxf(mx, rmx[(g & 1) * 256 + (1 - ewg) * 128 + r]);
+        bool need = false;
+        if (j == 0) {
+          c = M;
+        } else if (M > c + kTau) {
+          need = true;
+        }
+        if (__any_sync(0xffffffffu, need)) {  // raise this row's stabiliser: rescale O so far
+          mbar_wait(bar(C::B_SLOT + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, err);
+          tc_fence_after();
+          const float sc = need ? ex2(c - M) : 1.f;
+#pragma unroll
+          for (int cc = 0; cc < C::NR / 16; ++cc) {
+            const int col = C::T_O + ob * C::NR + ewg * (C::NR / 2) + 8 * cc;
+            uint32_t v[8];
+            tmem_ld8(taddr(tbase, eq, col), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * sc);
+            tmem_st8(taddr(tbase, eq, col), v);
+          }
+          tmem_wait_st();
+          if (need) c = M;
+        }
+        {  // phi in fp32, written back over the same columns this thread read
+          uint32_t w0[32], w1[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            w0[k] = __float_as_uint(ex2(u[k] - c));
+            w1[k] = __float_as_uint(ex2(u[32 + k] - c));
+          }
+          tmem_st32(taddr(tbase, eq, C::T_U + 128 * slot + 64 * ewg), w0);
+          tmem_st32(taddr(tbase, eq, C::T_U + 128 * slot + 64 * ewg + 32), w1);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_PHI + slot));
+      }
+      // ---- output tile: out = O[:, :d] / O[:, d] ----
+      mbar_wait(bar(C::B_OF + ob), (it >> 1) & 1, abort_flag, err);
+      tc_fence_after();
+      uint32_t num[D / 2];
+      uint32_t den;
+#pragma unroll
+      for (int h2 = 0; h2 < D / 64; ++h2) {
+        uint32_t t32[32];
+        tmem_ld32(taddr(tbase, eq, C::T_O + ob * C::NR + (D / 2) * ewg + 32 * h2), t32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) num[32 * h2 + k] = t32[k];
+      }
+      tmem_ld1(taddr(tbase, eq, C::T_O + ob * C::NR + D), den);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_OE + ob));
+      const float inv = 1.f / __uint_as_float(den);
+      const int T = T0 + it, bh = T / ntq, qt = T % ntq;
+      const int sb = it & 1;
+      if (issuer) bulk_wait_read<1>();
+      named_bar_sync(kBarStore, kEpiThreads);
+      // staging tile: 128 rows x D bf16, 64-dim regions of 128-byte rows, 128B swizzle
+#pragma unroll
+      for (int cc = 0; cc < D / 16; ++cc) {  // this thread's D/2 columns = D/16 chunks of 8
+        uint32_t w4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          w4[k] = pack_bf16x2(__uint_as_float(num[8 * cc + 2 * k]) * inv, __uint_as_float(num[8 * cc + 2 * k + 1]) * inv);
+        const int chunk = (D / 16) * ewg + cc;  // 16-byte chunk index within the D-wide row
+        const int rg = chunk >> 3, c8 = chunk & 7;
+        *reinterpret_cast<uint4*>(smem + C::S_OUT + sb * C::QTILE + rg * (128 * 128) + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(kBarStore, kEpiThreads);
+      if (issuer) {
+#pragma unroll
+        for (int rg = 0; rg < D / 64; ++rg)
+          tma_store_3d(&tmO, sbase + C::S_OUT + sb * C::QTILE + rg * (128 * 128), 64 * rg, qt * 128, bh);
+        bulk_commit();
+      }
+    }
+    if (issuer) bulk_wait<0>();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ============================================================================
+// Host side
+// ============================================================================
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [heads, L, d] bf16, boxes of 64 dims x 128 rows x 1 head, 128-byte swizzle; rows past L read as zero
+// and are not written.
+int make_map(CUtensorMap* map, const void* base, int d, int L, int heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return set_error(FAVOR_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_errorf(FAVOR_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FAVOR_OK;
+}
+
+int num_sms() {
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 1;
+}
+
+template <int D>
+int launch_key(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st) {
+  using C = KeyCfg<D>;
+  CUtensorMap mk, mv;
+  const int heads = p.B * p.Hkv;
+  int rc = make_map(&mk, K, D, p.L, heads);
+  if (rc == FAVOR_OK) rc = make_map(&mv, V, D, p.L, heads);
+  if (rc != FAVOR_OK) return rc;
+  auto kern = key_pass_sm100<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass attribute: %s", cudaGetErrorString(e));
+  char* base = static_cast<char*>(partials);
+  dim3 grid((p.m + 127) / 128, p.P, heads);
+  kern<<<grid, kThreads, C::SMEM, st>>>(mk, mv, W, reinterpret_cast<float*>(base + p.part_S_off),
+                                        reinterpret_cast<float*>(base + p.part_c_off), p.L, p.m, p.P, p.chunk,
+                                        p.nsb, p.wscale, p.nscale);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass launch: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
+template <int D>
+int launch_query(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st) {
+  using C = QueryCfg<D>;
+  CUtensorMap mq, mo;
+  const int bh = p.B * p.H;
+  int rc = make_map(&mq, Q, D, p.L, bh);
+  if (rc == FAVOR_OK) rc = make_map(&mo, out, D, p.L, bh);
+  if (rc != FAVOR_OK) return rc;
+  auto kern = query_pass_sm100<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass attribute: %s", cudaGetErrorString(e));
+  const int ntiles = bh * ((p.L + 127) / 128);
+  const int grid = ntiles < num_sms() ? ntiles : num_sms();
+  const unsigned char* img = static_cast<const unsigned char*>(state) + p.st_op_off;
+  kern<<<grid, kThreads, C::SMEM, st>>>(mq, mo, W, img, p.L, p.m, p.H, p.Hkv, ntiles, static_cast<int>(p.op_bytes),
+                                        p.wscale);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass launch: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
+}  // namespace
+
+bool sm100_key_supported(const Plan& p) { return p.d == 64 || p.d == 128; }
+bool sm100_query_supported(const Plan& p) { return p.d == 64 && p.m <= QueryCfg<64>::MMAX; }
+
+int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st) {
+  return p.d == 64 ? launch_key<64>(K, V, W, partials, p, st) : launch_key<128>(K, V, W, partials, p, st);
+}
+
+int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st) {
+  return launch_query<64>(Q, W, state, out, p, st);
+}
+
+int sm100_read_and_clear_error(unsigned int* word) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_sm100_error_word, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_sm100_error_word, &zero, sizeof(unsigned int));
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
+}  // namespace favor

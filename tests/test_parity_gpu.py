@@ -25,7 +25,7 @@ def f64(t):
 
 def gpu_attention(Q, K, V, W):
     out = fv.favor_attention(Q.cuda(), K.cuda(), V.cuda(), W.cuda())
-    torch.cuda.synchronize()
+    fv.favor_device_check()  # synchronises; raises if a kernel gave up waiting
     return out.cpu()
 
 
@@ -97,6 +97,34 @@ def test_growing_key_norms_force_rescaling():
     run_case(Q, (K * ramp).contiguous(), V, 128, what="ramp")
 
 
+def test_key_stabiliser_raised_late_bf16():
+    # the first key tiles have near-zero exponents; later keys sit on random feature rows,
+    # so their exponents are ~|w|^2/2 and the chunk stabiliser must be raised (and S rescaled)
+    d, m, L = 64, 256, 1500
+    W = fv.favor_make_features(1, m, d)
+    g = torch.Generator().manual_seed(7)
+    K = 0.01 * torch.randn(1, 1, L, d, generator=g)
+    rows = torch.randint(0, m, (L,), generator=g)
+    late = torch.arange(L) >= 300
+    K[0, 0, late] = W[rows[late]] * d ** 0.25 * 0.7
+    Q = torch.randn(1, 2, L, d, generator=g) * 0.5
+    V = torch.randn(1, 1, L, d, generator=g)
+    run_case(Q.bfloat16(), K.bfloat16(), V.bfloat16(), m, what="late keys")
+
+
+def test_query_stabiliser_raised_in_second_feature_block_bf16():
+    # each query sits on a feature row of the second 128-feature block, so its row max there
+    # exceeds the first block's and the running output must be rescaled
+    d, m, L = 64, 256, 700
+    W = fv.favor_make_features(1, m, d)
+    g = torch.Generator().manual_seed(8)
+    rows = torch.randint(128, m, (L,), generator=g)
+    Q = (W[rows] * d ** 0.25 * 0.6).view(1, 1, L, d).repeat(1, 2, 1, 1)
+    K = torch.randn(1, 1, L, d, generator=g)
+    V = torch.randn(1, 1, L, d, generator=g)
+    run_case(Q.bfloat16(), K.bfloat16(), V.bfloat16(), m, what="late queries")
+
+
 # ---- full sizes, in the launch configuration bench.py times ----------------
 def _full(name, orthogonal=True, heads=2, rows=256):
     w = wl.WORKLOADS[name]
@@ -135,7 +163,7 @@ def test_deterministic_bitwise():
     W = fv.favor_make_features(1, w.m, w.d).cuda()
     a = fv.favor_attention(Q, K, V, W)
     b = fv.favor_attention(Q, K, V, W)
-    torch.cuda.synchronize()
+    fv.favor_device_check()
     assert torch.equal(a, b)
 
 
@@ -152,16 +180,22 @@ def test_stage_calls_equal_fused_call_and_state_matches_oracle(dtype):
     out = torch.empty_like(Qd)
     fv.favor_query_pass(Qd, Wd, state, Hkv, out)
     fused = fv.favor_attention(Qd, Kd, Vd, Wd)
-    torch.cuda.synchronize()
+    fv.favor_device_check()
     assert torch.equal(out, fused)
     S, _ = fv.state_views(state, B, Hkv, d, m)
     Wo = ofv.make_features_f32(1, m, d)
+    # Each key feature carries a relative error of at most eps (bf16: 2^-9 rounding of phi
+    # plus ~1e-3 from the exponent argument; fp32: far below 1e-4), so every state entry
+    # sum_t phi_t v_t is within eps * sum_t phi_t |v_t| of the exact one.
+    eps = 6e-3 if dtype == torch.bfloat16 else 1e-4
     for b in range(B):
         for g in range(Hkv):
             So, _ = ofv.key_state(f64(K[b, g]), f64(V[b, g]), Wo)
+            Sa, _ = ofv.key_state(f64(K[b, g]), np.abs(f64(V[b, g])), Wo)
             Sg = S[b * Hkv + g].double().cpu().numpy()
             # the state is defined up to one positive constant (stabiliser, 1/sqrt(m))
-            np.testing.assert_allclose(Sg / Sg[:, d].sum(), So / So[:, d].sum(), rtol=1e-3, atol=1e-6)
+            gn, on = Sg / Sg[:, d].sum(), So / So[:, d].sum()
+            assert np.all(np.abs(gn - on) <= eps * Sa / So[:, d].sum() + 1e-12), np.abs(gn - on).max()
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
