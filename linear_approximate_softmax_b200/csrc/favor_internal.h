@@ -19,22 +19,24 @@ int make_features(uint64_t seed, int m, int d, int orthogonal, float* W_out);
 
 constexpr double kLog2e = 1.4426950408889634074;
 constexpr int kTileTokens = 128;   // key chunks are whole multiples of this
-constexpr int kStabBlock = 64;     // partial stabilisers are kept per 64 features
+constexpr int kStabBlock = 1;      // partial stabilisers are kept per feature
 
 // How the key pass splits each kv head's L tokens into P chunks.
 struct Plan {
   int B, H, Hkv, L, d, m;
   int P;            // chunks per kv head
   int chunk;        // tokens per chunk (multiple of kTileTokens, last one ragged)
-  int nsb;          // stabiliser blocks: ceil(m / kStabBlock)
+  int nsb;          // stabilisers per partial: ceil(m / kStabBlock) = m
   // byte offsets inside the partials buffer
   size_t part_S_off, part_c_off, part_bytes;
   // byte offsets inside the state buffer
   size_t st_S_off, st_c_off, st_op_off, st_bytes;
-  // The state re-packed as the fp32 (tf32) B operand of the query pass's
-  // second MMA: per kv head, op_atoms blocks of 32 features, each op_rows rows
-  // (output column n: d value columns, the normaliser at n = d, zeros after) of
-  // 128 B, K-major with the 128-byte swizzle (16-byte chunk c of row n at c ^ (n % 8)).
+  // The state re-packed as the fp16 B operand of the query pass's second MMA.
+  // Per kv head: op_atoms blocks of 64 features, each op_rows rows (output
+  // column n: d value columns, the normaliser at n = d, zeros after) of 128 B,
+  // K-major with the 128-byte swizzle (16-byte chunk c of row n at c ^ (n % 8));
+  // then e[64 * op_atoms] fp32.  Feature f's values are S[f][n] * 2^-e[f], with
+  // e[f] chosen so that the largest |S[f][n]| lands in [2^14, 2^15).
   int op_rows, op_atoms;
   size_t op_bytes;
   float wscale;     // d^-1/4 * log2(e): W is multiplied by this on the device

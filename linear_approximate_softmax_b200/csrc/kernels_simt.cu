@@ -18,6 +18,7 @@
 // the 1/sqrt(m) factors are constant along a query row and cancel exactly in
 // the ratio, as any per-row stabiliser does; they are not computed.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -28,7 +29,7 @@ namespace favor {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kFB = 64;   // features per key-pass CTA (== kStabBlock)
+constexpr int kFB = 64;   // features per key-pass CTA
 constexpr int kTT = 32;   // tokens per key-pass step
 constexpr int kQT = 32;   // queries per query-pass CTA
 
@@ -43,7 +44,8 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// grid (P, B*Hkv, ceil(m/64)), 256 threads.
+// grid (P, B*Hkv, ceil(m/64)), 256 threads.  One running stabiliser per CTA,
+// written for each of its features.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) key_pass_kernel(
     const T* __restrict__ K, const T* __restrict__ V, const float* __restrict__ W,
@@ -146,43 +148,73 @@ __global__ void __launch_bounds__(kThreads) key_pass_kernel(
       if (f < fbw) out[static_cast<size_t>(f0 + f) * D1 + c] = acc[k];
     }
   }
-  if (tid == 0) part_c[(static_cast<size_t>(head) * P + p) * nsb + fb] = c_run;
+  for (int f = tid; f < fbw; f += kThreads) part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + f] = c_run;
 }
 
-// grid (ceil(op_atoms*32*op_rows/256), B*Hkv), 256 threads.  One thread per
-// (feature f, column n) of the padded state: it sums the chunk partials in the
-// fixed order p = 0..P-1, each rescaled from its chunk stabiliser to the
-// largest one, writes S[f][n] (fp32) and the fp32 operand image of the query
-// pass (zeros in the padding).
+// grid (op_atoms * 64 / 32, B*Hkv), 256 threads: 32 feature rows per CTA, 8 threads
+// per row.  Each row is the sum of the chunk partials in the fixed order p = 0..P-1,
+// each rescaled from its own stabiliser to the head's largest one (bitwise
+// deterministic).  Writes S[f][n] (fp32), and the fp16 operand image of the query
+// pass: the row scaled by 2^-e[f] so that its largest entry lies in [2^14, 2^15)
+// (exact power-of-two scaling), zeros in the padding, and e[f].
 __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
     const float* __restrict__ part_S, const float* __restrict__ part_c, float* __restrict__ S,
     float* __restrict__ Sc, unsigned char* __restrict__ op, int P, int m, int D1, int nsb, int op_rows,
     int op_atoms, size_t op_bytes) {
+  __shared__ float red[kThreads / 32];
   const int head = blockIdx.y;
-  const int e = blockIdx.x * kThreads + threadIdx.x;
   const float* pc = part_c + static_cast<size_t>(head) * P * nsb;
-  float cs = -INFINITY;
-  for (int i = 0; i < P * nsb; ++i) cs = fmaxf(cs, pc[i]);
+  float cs = -INFINITY;  // the head's largest stabiliser
+  for (int i = threadIdx.x; i < P * nsb; i += kThreads) cs = fmaxf(cs, pc[i]);
+  cs = warp_max(cs);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = cs;
+  __syncthreads();
+  cs = red[0];
+#pragma unroll
+  for (int w = 1; w < kThreads / 32; ++w) cs = fmaxf(cs, red[w]);
   if (blockIdx.x == 0 && threadIdx.x == 0) Sc[head] = cs;
-  if (e >= op_atoms * 32 * op_rows) return;
-  const int f = e / op_rows, n = e % op_rows;
-  float val = 0.f;
-  if (f < m && n < D1) {
-    const int sb = f / kStabBlock;
-    const size_t idx = static_cast<size_t>(f) * D1 + n;
+
+  const int f = blockIdx.x * 32 + (threadIdx.x >> 3);  // feature row (< op_atoms * 64)
+  const int g = threadIdx.x & 7;                       // this thread's columns: g, g + 8, ...
+  constexpr int kMaxCols = (128 + 16) / 8;             // op_rows <= 144
+  float val[kMaxCols];
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < kMaxCols; ++k) {
+    const int n = g + 8 * k;
     float acc = 0.f;
-    for (int p = 0; p < P; ++p) {
-      const float c = pc[p * nsb + sb];
-      const float w = (c == -INFINITY) ? 0.f : exp2f(c - cs);
-      acc = fmaf(w, part_S[(static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * D1 + idx], acc);
+    if (n < op_rows && f < m && n < D1) {
+      const size_t idx = static_cast<size_t>(f) * D1 + n;
+      for (int p = 0; p < P; ++p) {
+        const float c = pc[p * nsb + f / kStabBlock];
+        const float wp = (c == -INFINITY) ? 0.f : exp2f(c - cs);
+        acc = fmaf(wp, part_S[(static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * D1 + idx], acc);
+      }
+      S[static_cast<size_t>(head) * m * D1 + idx] = acc;
     }
-    S[static_cast<size_t>(head) * m * D1 + idx] = acc;
-    val = acc;
+    val[k] = acc;
+    amax = fmaxf(amax, fabsf(acc));
   }
-  const int atom = f >> 5, chunk = (f & 31) >> 2, el = f & 3;
-  const size_t off = static_cast<size_t>(atom) * op_rows * 128 + static_cast<size_t>(n) * 128 +
-                     ((chunk ^ (n & 7)) << 4) + el * 4;
-  *reinterpret_cast<float*>(op + static_cast<size_t>(head) * op_bytes + off) = val;
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+  int ex = 0;
+  if (amax > 0.f) {
+    frexpf(amax, &ex);  // amax = mant * 2^ex, mant in [0.5, 1)
+    ex -= 15;           // amax * 2^-ex in [2^14, 2^15)
+  }
+  unsigned char* img = op + static_cast<size_t>(head) * op_bytes;
+  const int atom = f >> 6, chunk = (f & 63) >> 3, el = f & 7;
+#pragma unroll
+  for (int k = 0; k < kMaxCols; ++k) {
+    const int n = g + 8 * k;
+    if (n < op_rows) {
+      const size_t off = static_cast<size_t>(atom) * op_rows * 128 + static_cast<size_t>(n) * 128 +
+                         ((chunk ^ (n & 7)) << 4) + el * 2;
+      *reinterpret_cast<__half*>(img + off) = __float2half_rn(ldexpf(val[k], -ex));
+    }
+  }
+  if (g == 0) reinterpret_cast<float*>(img + static_cast<size_t>(op_rows) * 128 * op_atoms)[f] = static_cast<float>(ex);
 }
 
 // grid (ceil(L/32), B*H), 256 threads.
@@ -315,7 +347,7 @@ int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void*
 int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int D1 = p.d + 1;
-  dim3 grid((p.op_atoms * 32 * p.op_rows + kThreads - 1) / kThreads, p.B * p.Hkv);
+  dim3 grid(p.op_atoms * 64 / 32, p.B * p.Hkv);
   const char* pb = static_cast<const char*>(partials);
   char* sb = static_cast<char*>(state);
   state_reduce_kernel<<<grid, kThreads, 0, st>>>(

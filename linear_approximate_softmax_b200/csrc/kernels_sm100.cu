@@ -17,13 +17,15 @@
 //
 // Query pass (one CTA per SM over a contiguous range of 128-query tiles):
 //   MMA1  U[q, f] = Q[q, :] . W'[f, :]        A = Q tile (TMA), B = W' hi + lo (smem), per 128-feature block
-//   exp   phi[q, f] = 2^(U - c_q)             fp32, written back over U; c_q = the row max,
+//   exp   phi'[q, f] = 2^(U + e_f - c_q)      fp16, written back over U; c_q = the row max of U + e,
 //                                             raised lazily across feature blocks
-//   MMA2  O[q, :] += phi[q, block] . S'[block, :]   kind::tf32: A = phi in TMEM, B = fp32 state image (smem)
+//   MMA2  O[q, :] += phi'[q, block] . S'[block, :]   kind::f16: A = phi' in TMEM, B = fp16 state image
 //   out = O[:, :d] / O[:, d] -> bf16 -> TMA store.
-// MMA2 runs in tf32 rather than bf16 because rounding the state to bf16 costs up to
-// 2^-8 of an output when one feature dominates a query, which, with the bf16 output
-// rounding on top, reaches the 2e-2 max-abs bound.
+// The state image holds each feature row scaled by its own power of two, S' = 2^-e_f S,
+// so that fp16 keeps 11 bits for every row; adding e_f to the exponent restores the
+// product exactly.  bf16 operands (8 bits) cost up to 2^-8 of an output when one
+// feature dominates a query, which, with the bf16 output rounding, reaches the 2e-2
+// max-abs bound; tf32 would need twice the MMA instructions.
 //
 // W' = d^-1/4 log2(e) W is split as W' = hi + lo in bf16 so that the exponent
 // arguments keep ~17 bits: a single bf16 W' moves the exponents by up to
@@ -48,15 +50,28 @@ __device__ unsigned int g_sm100_error_word;
 namespace {
 using namespace sm100;
 
-constexpr int kThreads = 384;  // 12 warps: producer, MMA, two spare/norm warps, 8 epilogue warps
+constexpr int kThreads = 384;  // key pass: producer, MMA, two norm warps, 8 epilogue warps
 constexpr int kEpiWarp0 = 4;
 constexpr int kEpiThreads = 256;
-constexpr uint32_t kBarEpi = 1;    // named barrier: epilogue max exchange
-constexpr uint32_t kBarStore = 2;  // named barrier: output staging
+constexpr uint32_t kBarEpi = 1;    // named barrier: epilogue max exchange (lock-step key pass)
 constexpr float kTau = 8.f;        // lazy stabiliser threshold (log2 units)
 
 __device__ __forceinline__ uint32_t taddr(uint32_t base, int lane_quarter, int col) {
   return base + (static_cast<uint32_t>(lane_quarter * 32) << 16) + static_cast<uint32_t>(col);
+}
+
+// Multiplies `chunks` x 8 consecutive TMEM columns of this warp's 32 lanes by `sc` (per lane).
+// A cold path (a raised stabiliser), kept out of line so it costs the hot loop no registers.
+__device__ __noinline__ void scale_tmem_row(uint32_t taddr0, int chunks, float sc) {
+  for (int cc = 0; cc < chunks; ++cc) {
+    uint32_t v[8];
+    tmem_ld8(taddr0 + 8 * cc, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * sc);
+    tmem_st8(taddr0 + 8 * cc, v);
+  }
+  tmem_wait_st();
 }
 
 // ============================================================================
@@ -97,7 +112,9 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
     float nscale) {
   using C = KeyCfg<D>;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // offset the __shared__ array itself (not via an integer cast), so that every pointer derived
+  // from it stays a shared-memory pointer and compiles to shared loads and stores
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // the feature groups of one (kv head, chunk) are adjacent CTAs, so they run together and the
@@ -370,10 +387,310 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
           if (col0 + k <= D) outp[static_cast<size_t>(f0 + frow) * (D + 1) + col0 + k] = __uint_as_float(v[k]);
       }
     }
-    if (warp == kEpiWarp0 && lane == 0) {
-      for (int sb = 2 * grp; sb < min(nsb, 2 * grp + 2); ++sb)
-        part_c[(static_cast<size_t>(head) * P + p) * nsb + sb] = c_run;
+    if (ewg == 0 && fvalid) part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + frow] = c_run;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ============================================================================
+// Key pass, d = 64: the two epilogue warpgroups take alternate tiles
+// ============================================================================
+// Each warpgroup owns one U^T buffer, one S accumulator, its own running
+// stabiliser and its own MMA-issuing thread (warp 1 for warpgroup 0, warp 2 for
+// warpgroup 1), so one warpgroup's exp work overlaps the other's TMEM loads and
+// MMAs.  A warpgroup computes the key norms of its next tile itself, between
+// handing phi to its MMA2 and the arrival of its next U^T.  At the end the two
+// accumulators are merged exactly: S = 2^(c0-c) S0 + 2^(c1-c) S1.
+struct KeyPP {
+  static constexpr int D = 64;
+  static constexpr int NST = 4;
+  static constexpr int TILE = 128 * 64 * 2;
+  static constexpr int NS = D + 16;
+  static constexpr int T_WHI = 0, T_WLO = 32, T_D1 = 64, T_S = 64 + 256;  // S[w] at T_S + NS*w
+  static_assert(T_S + 2 * NS <= 512, "TMEM budget");
+  static constexpr int S_K = 0;
+  static constexpr int S_V = S_K + NST * TILE;
+  // [V | 1] as one N = 80 MN-major operand: the ones column is the first column of a
+  // second 64-column atom, LBO bytes after the V tile of the stage
+  static constexpr int S_ONES = S_V + NST * TILE;  // 128 tokens x 64 columns, column 0 = 1
+  static constexpr int S_NRM = S_ONES + TILE;
+  static constexpr int S_CW = S_NRM + NST * 512;   // final stabilisers, [warpgroup][feature]
+  static constexpr int S_BAR = S_CW + 1024;
+  static constexpr int B_KVF = 0, B_KVE = 4, B_D1F = 8, B_PHI = 10, B_SDONE = 12, NBAR = 14;
+  static constexpr int S_TPTR = S_BAR + NBAR * 8;
+  static constexpr int S_ABORT = S_TPTR + 8;
+  static constexpr int SMEM = S_ABORT + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const float* __restrict__ W,
+    float* __restrict__ part_S, float* __restrict__ part_c, int L, int m, int P, int chunk, int nsb, float wscale,
+    float nscale) {
+  using C = KeyPP;
+  constexpr int D = C::D;
+  extern __shared__ unsigned char smem_raw[];
+  // offset the __shared__ array itself (not via an integer cast), so that every pointer derived
+  // from it stays a shared-memory pointer and compiles to shared loads and stores
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = blockIdx.x, p = blockIdx.y, head = blockIdx.z;
+  const int f0 = grp * 128, gw = min(128, m - f0);
+  const int t_begin = p * chunk, t_end = min(L, t_begin + chunk);
+  const int ntiles = (t_end - t_begin + 127) / 128;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
+  uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
+  float* nrm = reinterpret_cast<float*>(smem + C::S_NRM);
+  float* cw = reinterpret_cast<float*>(smem + C::S_CW);
+  auto bar = [&](int i) { return sbase + C::S_BAR + 8u * i; };
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(bar(C::B_KVF + s), 1);
+      mbar_init(bar(C::B_KVE + s), 1);
     }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(bar(C::B_D1F + w), 1);
+      mbar_init(bar(C::B_PHI + w), 4);
+      mbar_init(bar(C::B_SDONE + w), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tptr_slot), 512);
+    tmem_relinquish();
+  }
+  for (int i = tid; i < C::TILE / 4; i += kThreads) {  // ones atom: row t, logical column 0 = 1.0
+    const int t = i / 32, word = i % 32;                  // 32 words per 128-byte row
+    // logical chunk 0 of row t sits at physical chunk (t % 8) under the 128-byte swizzle
+    reinterpret_cast<uint32_t*>(smem + C::S_ONES)[i] = (word == (t & 7) * 4) ? 0x00003F80u : 0u;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tptr_slot;
+
+  const bool epi = warp >= kEpiWarp0;
+  const int eq = warp & 3;
+  const int ewg = (warp - kEpiWarp0) >> 2;
+  const int frow = eq * 32 + lane;
+  const bool fvalid = frow < gw;
+
+  if (epi) {  // W' hi (warpgroup 0) / lo (warpgroup 1) into TMEM, lane = feature
+    const int f = f0 + frow;
+    uint32_t words[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float w0 = 0.f, w1 = 0.f;
+      if (fvalid) {
+        const float2 v = *reinterpret_cast<const float2*>(W + static_cast<size_t>(f) * D + 2 * j);
+        w0 = v.x * wscale;
+        w1 = v.y * wscale;
+      }
+      if (ewg == 0) {
+        words[j] = pack_bf16x2(w0, w1);
+      } else {
+        const float h0 = __bfloat162float(__float2bfloat16_rn(w0));
+        const float h1 = __bfloat162float(__float2bfloat16_rn(w1));
+        words[j] = pack_bf16x2(w0 - h0, w1 - h1);
+      }
+    }
+    tmem_st32(taddr(tbase, eq, ewg == 0 ? C::T_WHI : C::T_WLO), words);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  unsigned int* err = &g_sm100_error_word;
+  const int cnt_of[2] = {(ntiles + 1) / 2, ntiles / 2};  // tiles of each warpgroup
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % C::NST;
+        if (i >= C::NST && !mbar_wait(bar(C::B_KVE + s), ((i / C::NST) - 1) & 1, abort_flag, err)) break;
+        mbar_arrive_expect_tx(bar(C::B_KVF + s), 2 * C::TILE);
+        const int t0 = t_begin + 128 * i;
+        tma_load_3d(sbase + C::S_K + s * C::TILE, &tmK, bar(C::B_KVF + s), 0, t0, head);
+        tma_load_3d(sbase + C::S_V + s * C::TILE, &tmV, bar(C::B_KVF + s), 0, t0, head);
+        issued = i + 1;
+      }
+      for (int i = max(0, issued - C::NST); i < issued; ++i)
+        mbar_wait(bar(C::B_KVF + i % C::NST), (i / C::NST) & 1, abort_flag, err, 200000000ull);
+    }
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers: warp 1 serves warpgroup 0, warp 2 warpgroup 1 ----------------
+    // One issuing thread per warpgroup, each in tile order, so neither warpgroup's MMAs
+    // wait behind the other's in a shared issue loop.
+    if (lane == 0) {
+      const int w = warp - 1;
+      const uint32_t id1 = idesc_bf16(128, 128, false, false);
+      const uint32_t idv = idesc_bf16(128, C::NS, false, true);  // N = 80: V, then the ones column
+      const uint32_t d1 = tbase + C::T_D1 + 128 * w;
+      const uint32_t sw = tbase + C::T_S + C::NS * w;
+      int cnt = 0;
+      for (int i = w; i < ntiles; i += 2, ++cnt) {
+        const int s = i % C::NST;
+        if (!mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err)) break;
+        if (cnt >= 1 && !mbar_wait(bar(C::B_SDONE + w), (cnt - 1) & 1, abort_flag, err)) break;  // U^T buffer free
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {  // MMA1: U^T = W' K^T (hi, then lo)
+          const uint64_t bk = sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * ks, 16, 1024);
+          mma_ts(d1, tbase + C::T_WHI + 8 * ks, bk, id1, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t bk = sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * ks, 16, 1024);
+          mma_ts(d1, tbase + C::T_WLO + 8 * ks, bk, id1, 1u);
+        }
+        mma_commit(bar(C::B_D1F + w));
+        if (!mbar_wait(bar(C::B_PHI + w), cnt & 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t lbo = C::S_ONES - (C::S_V + s * C::TILE);  // V atom -> ones atom
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {  // MMA2: S_w += phi^T [V | 1]
+          const uint64_t bv = sdesc_sw128(sbase + C::S_V + s * C::TILE + 2048 * ks, lbo, 1024);
+          mma_ts(sw, d1 + 8 * ks, bv, idv, (cnt > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(C::B_KVE + s));
+        mma_commit(bar(C::B_SDONE + w));
+      }
+      const int mine = (ntiles + 1 - w) / 2;
+      if (mine > 0) mbar_wait(bar(C::B_SDONE + w), (mine - 1) & 1, abort_flag, err, 200000000ull);
+    }
+  } else if (epi) {
+    // ---------------- epilogue warpgroup ewg: tiles ewg, ewg + 2, ... ----------------
+    // Each thread owns feature f0 + frow and reads each U^T value of its row once.  Its
+    // stabiliser c is that feature's running max exponent over the tiles seen so far,
+    // raised (with an exact rescale of its S row) only when a tile exceeds it by more
+    // than 2^kTau, and never below floor = |w|^2 log2(e)/2 - 64: by completing the square
+    // no exponent of this feature exceeds |w|^2 log2(e)/2, so no phi exceeds 2^64 and the
+    // fp32 state cannot overflow for any |v| < 2^46 at any sequence length up to 2^17.
+    float floor_c;
+    {
+      float w2 = 0.f;
+      if (fvalid) {
+        const float4* wr = reinterpret_cast<const float4*>(W + static_cast<size_t>(f0 + frow) * D);
+#pragma unroll
+        for (int k = 0; k < D / 4; ++k) {
+          const float4 v = wr[k];
+          w2 = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, w2))));
+        }
+      }
+      floor_c = w2 * static_cast<float>(kLog2e * 0.5) - 64.f;
+    }
+    float c_run = floor_c, tmax = -INFINITY;
+    const uint32_t d1col = C::T_D1 + 128 * ewg;
+    const uint32_t scol = C::T_S + C::NS * ewg;
+    // n(k) = |k|^2 * nscale of tile i's key frow (this thread's token), +inf past the chunk end;
+    // the 16-byte chunks of a swizzled row are summed in any order
+    auto key_norms = [&](int i) {
+      const int s = i % C::NST;
+      mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err);
+      const uint4* row = reinterpret_cast<const uint4*>(smem + C::S_K + s * C::TILE + frow * 128);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = row[c];
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float lo = __uint_as_float(wv[k] << 16), hi = __uint_as_float(wv[k] & 0xFFFF0000u);
+          acc[k] = fmaf(lo, lo, acc[k]);
+          acc[k] = fmaf(hi, hi, acc[k]);
+        }
+      }
+      const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      nrm[s * 128 + frow] = (t_begin + 128 * i + frow < t_end) ? sum * nscale : INFINITY;
+      named_bar_sync(1 + ewg, 128);  // the warpgroup's 128 norms are in shared memory
+    };
+    int cnt = 0;
+    if (ewg < ntiles) key_norms(ewg);
+    for (int i = ewg; i < ntiles; i += 2, ++cnt) {
+      const int s = i % C::NST;
+      mbar_wait(bar(C::B_D1F + ewg), cnt & 1, abort_flag, err);
+      tc_fence_after();
+      // the previous tile raised the running max: rescale S now (its MMA2 has completed,
+      // since this tile's MMA1 was issued after it)
+      const bool need = tmax > c_run + kTau;
+      if (__any_sync(0xffffffffu, need)) scale_tmem_row(taddr(tbase, eq, scol), C::NS / 8, need ? ex2(c_run - tmax) : 1.f);
+      if (need) c_run = tmax;
+      const float cc_run = c_run;
+      const float4* nv = reinterpret_cast<const float4*>(nrm + s * 128);
+      uint32_t cur[32], nxt[32];
+      tmem_ld32(taddr(tbase, eq, d1col), cur);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        if (q4 < 3) tmem_ld32(taddr(tbase, eq, d1col + 32 * (q4 + 1)), nxt);  // next chunk streams in meanwhile
+        uint32_t wph[16];
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 n4 = nv[8 * q4 + k4];
+          const float a0 = __uint_as_float(cur[4 * k4 + 0]) - n4.x;
+          const float a1 = __uint_as_float(cur[4 * k4 + 1]) - n4.y;
+          const float a2 = __uint_as_float(cur[4 * k4 + 2]) - n4.z;
+          const float a3 = __uint_as_float(cur[4 * k4 + 3]) - n4.w;
+          tmax = max3(tmax, a0, a1);
+          tmax = max3(tmax, a2, a3);
+          wph[2 * k4] = pack_bf16x2(ex2(a0 - cc_run), ex2(a1 - cc_run));
+          wph[2 * k4 + 1] = pack_bf16x2(ex2(a2 - cc_run), ex2(a3 - cc_run));
+        }
+        if (!fvalid) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) wph[k] = 0u;
+        }
+        tmem_st16(taddr(tbase, eq, d1col + 16 * q4), wph);  // phi over columns already read
+        if (q4 < 3) {
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) cur[k] = nxt[k];
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_PHI + ewg));
+      if (i + 2 < ntiles) key_norms(i + 2);  // while this tile's MMA2 and the next MMA1 run
+    }
+    // merge the two accumulators row by row and write this group's partial state
+    cw[ewg * 128 + frow] = c_run;
+    named_bar_sync(3, kEpiThreads);
+    const float c0 = cw[frow], c1 = cw[128 + frow];
+    const bool has1 = cnt_of[1] > 0;
+    const float cmax = has1 ? fmaxf(c0, c1) : c0;
+    mbar_wait(bar(C::B_SDONE + 0), (cnt_of[0] - 1) & 1, abort_flag, err);
+    if (has1) mbar_wait(bar(C::B_SDONE + 1), (cnt_of[1] - 1) & 1, abort_flag, err);
+    tc_fence_after();
+    const float s0 = ex2(c0 - cmax), s1 = has1 ? ex2(c1 - cmax) : 0.f;
+    float* outp = part_S + (static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * (D + 1);
+#pragma unroll
+    for (int cc = 0; cc < C::NS / 16; ++cc) {  // this warpgroup's half of the columns
+      const int col0 = ewg * (C::NS / 2) + 8 * cc;
+      uint32_t v0[8], v1[8];
+      tmem_ld8(taddr(tbase, eq, C::T_S + col0), v0);
+      tmem_ld8(taddr(tbase, eq, C::T_S + C::NS + col0), v1);
+      tmem_wait_ld();
+      if (fvalid) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float v = __uint_as_float(v0[k]) * s0;
+          if (has1) v = fmaf(__uint_as_float(v1[k]), s1, v);
+          if (col0 + k <= D) outp[static_cast<size_t>(f0 + frow) * (D + 1) + col0 + k] = v;
+        }
+      }
+    }
+    if (ewg == 0 && fvalid) part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + frow] = cmax;
   }
   tc_fence_before();
   __syncthreads();
@@ -386,73 +703,78 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
 // ============================================================================
 template <int D>
 struct QueryCfg {
-  static constexpr int NSTQ = 2;
+  static constexpr int THREADS = 256;  // producer, MMA, two idle warps, one epilogue warpgroup (warps 4-7)
   static constexpr int QTILE = 128 * D * 2;
   static constexpr int NR = D + 16;                  // output columns of MMA2 (values, normaliser, zeros)
   static constexpr int MMAX = 256;                   // features held in shared memory
-  static constexpr int SP = NR * 128 * (MMAX / 32);  // the fp32 state image (one buffer)
+  static constexpr int SP = NR * 128 * (MMAX / 64) + 4 * MMAX;  // fp16 state image + exponents (one buffer)
+  static constexpr int NU = 3;                       // U buffers: MMA1 runs up to two blocks ahead
   // TMEM columns
-  static constexpr int T_U = 0;        // 2 slots x 128
-  static constexpr int T_O = 256;      // 2 buffers x NR
-  static_assert(T_O + 2 * NR <= 512, "TMEM budget");
+  static constexpr int T_U = 0;          // NU x 128
+  static constexpr int T_O = NU * 128;   // NR
+  static_assert(T_O + NR <= 512, "TMEM budget");
   // shared memory
   static constexpr int S_WHI = 0;
   static constexpr int S_WLO = S_WHI + MMAX * 128 * (D / 64);
   static constexpr int S_SP = S_WLO + MMAX * 128 * (D / 64);
-  static constexpr int S_Q = S_SP + SP;
-  static constexpr int S_OUT = S_Q + NSTQ * QTILE;
-  static constexpr int S_RMX = S_OUT + 2 * QTILE;   // 2 x 2 x 128 floats
-  static constexpr int S_BAR = S_RMX + 2048;
-  // barriers
-  static constexpr int B_QF = 0, B_QE = 2, B_SF = 4, B_SE = 6, B_UF = 8, B_PHI = 10, B_SLOT = 12, B_OF = 14,
-                       B_OE = 16, NBAR = 18;
+  static constexpr int S_Q = S_SP + SP;               // 2 stages, by tile parity
+  static constexpr int S_OUT = S_Q + 2 * QTILE;       // output staging
+  static constexpr int S_BAR = S_OUT + QTILE;
+  static constexpr int B_QF = 0, B_QE = 2, B_UF = 4, B_PHI = 7, B_M2 = 10, B_OF = 13, B_OE = 14, B_SF = 15,
+                       B_SE = 16, NBAR = 17;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int SMEM = S_ABORT + 16 + 1024;
 };
 
-struct QueryRange {
-  int T0, T1;  // tiles [T0, T1) of this CTA
-};
-
+// Query pass: one epilogue warpgroup; each thread owns one query row and holds a whole
+// 128-feature block of it in registers, so every U value is read from tensor memory once
+// and the row max is exact.  While it exponentiates block g it streams block g+1 in.
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) query_pass_sm100(
+__global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, const float* __restrict__ W,
     const unsigned char* __restrict__ op_img, int L, int m, int H, int Hkv, int ntiles_total, int op_bytes,
     float wscale) {
   using C = QueryCfg<D>;
+  constexpr int NT = C::THREADS;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // offset the __shared__ array itself (not via an integer cast), so that every pointer derived
+  // from it stays a shared-memory pointer and compiles to shared loads and stores
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ntq = (L + 127) / 128;
   const int G = H / Hkv;
   const int nb = (m + 127) / 128;
-  // contiguous, balanced range of tiles for this CTA
   const int per = ntiles_total / gridDim.x, extra = ntiles_total % gridDim.x;
   const int T0 = blockIdx.x * per + min(static_cast<int>(blockIdx.x), extra);
   const int n = per + (static_cast<int>(blockIdx.x) < extra ? 1 : 0);
+  const int nblk = n * nb;  // blocks of this CTA, tile-major
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
   uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
-  float* rmx = reinterpret_cast<float*>(smem + C::S_RMX);
   auto bar = [&](int i) { return sbase + C::S_BAR + 8u * i; };
+  // kv head of a tile; non-decreasing along the tile order, so the CTA's tiles visit each
+  // kv head once and the image index of local tile it is kvh_of(T0 + it) - kvh_of(T0)
   auto kvh_of = [&](int T) {
     const int bh = T / ntq;
     return (bh / H) * Hkv + (bh % H) / G;
   };
+  const int kvh0 = kvh_of(T0);
 
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(C::B_QF + i), 1);
       mbar_init(bar(C::B_QE + i), 1);
-      mbar_init(bar(C::B_SF + i), 1);
-      mbar_init(bar(C::B_SE + i), 1);
-      mbar_init(bar(C::B_UF + i), 1);
-      mbar_init(bar(C::B_PHI + i), kEpiThreads / 32);
-      mbar_init(bar(C::B_SLOT + i), 1);
-      mbar_init(bar(C::B_OF + i), 1);
-      mbar_init(bar(C::B_OE + i), kEpiThreads / 32);
     }
+    for (int i = 0; i < C::NU; ++i) {
+      mbar_init(bar(C::B_UF + i), 1);
+      mbar_init(bar(C::B_PHI + i), 4);
+      mbar_init(bar(C::B_M2 + i), 1);
+    }
+    mbar_init(bar(C::B_OF), 1);
+    mbar_init(bar(C::B_OE), 4);
+    mbar_init(bar(C::B_SF), 1);
+    mbar_init(bar(C::B_SE), 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmQ);
@@ -466,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1) query_pass_sm100(
   {
     const int rows = nb * 128;
     constexpr int CPR = D / 8;  // 16-byte chunks per row
-    for (int item = tid; item < rows * CPR; item += kThreads) {
+    for (int item = tid; item < rows * CPR; item += NT) {
       const int f = item / CPR, c = item % CPR;
       const int rg = c >> 3, cc = c & 7;  // 64-dim region, chunk within the 128-byte row
       uint32_t hi[4], lo[4];
@@ -495,217 +817,223 @@ __global__ void __launch_bounds__(kThreads, 1) query_pass_sm100(
   unsigned int* err = &g_sm100_error_word;
 
   if (warp == 0) {
-    // ---------------- producer: state images and Q tiles ----------------
+    // ---------------- producer: Q tiles (2 stages) and state images ----------------
     if (lane == 0) {
-      int k = -1, prev = -1, issued = 0;
+      int loaded = -1, issued = 0;
       for (int it = 0; it < n; ++it) {
-        const int T = T0 + it;
-        // the Q tile first: the MMA warp issues the previous head's last MMA2 (which releases
-        // the state image) only after this tile's first MMA1
-        const int s = it % C::NSTQ;
-        if (it >= C::NSTQ && !mbar_wait(bar(C::B_QE + s), ((it / C::NSTQ) - 1) & 1, abort_flag, err)) break;
+        const int T = T0 + it, s = it & 1;
+        // the Q tile first: the previous image is released only after this tile's MMA1s
+        if (it >= 2 && !mbar_wait(bar(C::B_QE + s), ((it >> 1) - 1) & 1, abort_flag, err)) break;
         mbar_arrive_expect_tx(bar(C::B_QF + s), C::QTILE);
         const int bh = T / ntq, qt = T % ntq;
 #pragma unroll
         for (int r = 0; r < D / 64; ++r)
           tma_load_3d(sbase + C::S_Q + s * C::QTILE + r * (128 * 128), &tmQ, bar(C::B_QF + s), 64 * r, qt * 128, bh);
         issued = it + 1;
-        const int kvh = kvh_of(T);
-        if (kvh != prev) {  // new kv head: its state image replaces the previous one once that is released
-          ++k;
-          prev = kvh;
+        const int k = kvh_of(T) - kvh0;
+        if (k > loaded) {  // a new kv head: load its image once the previous one is released
           if (k >= 1 && !mbar_wait(bar(C::B_SE), (k - 1) & 1, abort_flag, err)) break;
           mbar_arrive_expect_tx(bar(C::B_SF), op_bytes);
-          bulk_load(sbase + C::S_SP, op_img + static_cast<size_t>(kvh) * op_bytes, op_bytes, bar(C::B_SF));
+          bulk_load(sbase + C::S_SP, op_img + static_cast<size_t>(kvh0 + k) * op_bytes, op_bytes, bar(C::B_SF));
+          loaded = k;
         }
       }
-      for (int it = max(0, issued - C::NSTQ); it < issued; ++it)
-        mbar_wait(bar(C::B_QF + it % C::NSTQ), (it / C::NSTQ) & 1, abort_flag, err, 200000000ull);
-      if (k >= 0) mbar_wait(bar(C::B_SF), k & 1, abort_flag, err, 200000000ull);
+      for (int it = max(0, issued - 2); it < issued; ++it)
+        mbar_wait(bar(C::B_QF + (it & 1)), (it >> 1) & 1, abort_flag, err, 200000000ull);
+      if (loaded >= 0) mbar_wait(bar(C::B_SF), loaded & 1, abort_flag, err, 200000000ull);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+    // ---------------- MMA issuer: MMA1 up to two blocks ahead of MMA2 ----------------
     if (lane == 0) {
-      const uint32_t id2 = idesc_tf32(128, C::NR, false, false);
-      int k = -1, prev = -1;  // state image index of the tile whose MMA2s are being issued
-      auto mma2 = [&](int h) {
-        const int it = h / nb, j = h % nb, slot = h & 1, ob = it & 1;
-        if (!mbar_wait(bar(C::B_PHI + slot), (h >> 1) & 1, abort_flag, err)) return false;
-        if (j == 0) {
-          if (it >= 2 && !mbar_wait(bar(C::B_OE + ob), ((it >> 1) - 1) & 1, abort_flag, err)) return false;
-          const int kvh = kvh_of(T0 + it);
-          if (kvh != prev) {
-            ++k;
-            prev = kvh;
-            if (!mbar_wait(bar(C::B_SF), k & 1, abort_flag, err)) return false;
-          }
-        }
-        tc_fence_after();
-        const int bw = min(128, m - 128 * j);
-        for (int ks = 0; ks < bw / 8; ++ks) {  // tf32: 8 features per step, one TMEM column each
-          const int fk = 128 * j + 8 * ks;
-          const uint64_t bd = sdesc_sw128(sbase + C::S_SP + (fk >> 5) * (C::NR * 128) + 32 * ((fk & 31) >> 3), 16, 1024);
-          mma_ts_tf32(tbase + C::T_O + ob * C::NR, tbase + C::T_U + 128 * slot + 8 * ks, bd, id2,
-                      (j > 0 || ks > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(C::B_SLOT + slot));
-        if (j == nb - 1) {
-          mma_commit(bar(C::B_OF + ob));
-          if (it == n - 1 || kvh_of(T0 + it + 1) != prev) mma_commit(bar(C::B_SE));
-        }
-        return true;
-      };
+      const uint32_t id2 = idesc_f16(128, C::NR, false, false);
+      int a = 0;  // next block for MMA1
       bool ok = true;
-      int g = 0;
-      for (int it = 0; it < n && ok; ++it) {
-        const int s = it % C::NSTQ;
-        for (int j = 0; j < nb && ok; ++j, ++g) {
-          const int slot = g & 1;
-          if (j == 0 && !mbar_wait(bar(C::B_QF + s), (it / C::NSTQ) & 1, abort_flag, err)) { ok = false; break; }
-          if (g >= 2 && !mbar_wait(bar(C::B_SLOT + slot), ((g >> 1) - 1) & 1, abort_flag, err)) { ok = false; break; }
+      for (int b = 0; b < nblk && ok; ++b) {  // MMA2 of block b
+        while (a < nblk && a < b + C::NU) {
+          const int ta = a / nb, ja = a % nb, sa = a % C::NU;
+          if (ja == 0 && !mbar_wait(bar(C::B_QF + (ta & 1)), (ta >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          if (a >= C::NU && !mbar_wait(bar(C::B_M2 + sa), ((a / C::NU) - 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          const int bw = min(128, m - 128 * j);
+          const int bw = min(128, m - 128 * ja);
           const uint32_t id1 = idesc_bf16(128, bw, false, false);
-          const uint32_t dU = tbase + C::T_U + 128 * slot;
+          const uint32_t dU = tbase + C::T_U + 128 * sa;
+          const uint32_t qbase = sbase + C::S_Q + (ta & 1) * C::QTILE;
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
             const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
-            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * j) * 128 + 32 * (ks & 3);
-            mma_ss(dU, sdesc_sw128(sbase + C::S_Q + s * C::QTILE + qo, 16, 1024),
-                   sdesc_sw128(sbase + C::S_WHI + wo, 16, 1024), id1, ks > 0 ? 1u : 0u);
+            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * ja) * 128 + 32 * (ks & 3);
+            mma_ss(dU, sdesc_sw128(qbase + qo, 16, 1024), sdesc_sw128(sbase + C::S_WHI + wo, 16, 1024), id1,
+                   ks > 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
             const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
-            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * j) * 128 + 32 * (ks & 3);
-            mma_ss(dU, sdesc_sw128(sbase + C::S_Q + s * C::QTILE + qo, 16, 1024),
-                   sdesc_sw128(sbase + C::S_WLO + wo, 16, 1024), id1, 1u);
+            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * ja) * 128 + 32 * (ks & 3);
+            mma_ss(dU, sdesc_sw128(qbase + qo, 16, 1024), sdesc_sw128(sbase + C::S_WLO + wo, 16, 1024), id1, 1u);
           }
-          mma_commit(bar(C::B_UF + slot));
-          if (j == nb - 1) mma_commit(bar(C::B_QE + s));
-          if (g >= 1) ok = mma2(g - 1);
+          mma_commit(bar(C::B_UF + sa));
+          if (ja == nb - 1) mma_commit(bar(C::B_QE + (ta & 1)));
+          ++a;
         }
-      }
-      if (ok && g >= 1 && !*abort_flag) mma2(g - 1);
-      if (g >= 1) mbar_wait(bar(C::B_SLOT + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, err, 200000000ull);
-    }
-  } else if (warp >= kEpiWarp0) {
-    // ---------------- epilogue ----------------
-    const int eq = warp & 3, ewg = (warp - kEpiWarp0) >> 2;
-    const int r = eq * 32 + lane;  // query row within the tile (TMEM lane)
-    const bool issuer = (warp == kEpiWarp0 && lane == 0);
-    int g = 0;
-    for (int it = 0; it < n; ++it) {
-      const int ob = it & 1;
-      float c = -INFINITY;
-      for (int j = 0; j < nb; ++j, ++g) {
-        const int slot = g & 1;
-        mbar_wait(bar(C::B_UF + slot), (g >> 1) & 1, abort_flag, err);
+        if (!ok) break;
+        const int tb = b / nb, jb = b % nb, sb = b % C::NU;
+        if (!mbar_wait(bar(C::B_PHI + sb), (b / C::NU) & 1, abort_flag, err)) break;
+        const int k = kvh_of(T0 + tb) - kvh0;
+        if (jb == 0) {
+          if (tb >= 1 && !mbar_wait(bar(C::B_OE), (tb - 1) & 1, abort_flag, err)) break;
+          if (!mbar_wait(bar(C::B_SF), k & 1, abort_flag, err)) break;
+        }
         tc_fence_after();
-        float u[64];
-        {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(taddr(tbase, eq, C::T_U + 128 * slot + 64 * ewg), r0);
-          tmem_ld32(taddr(tbase, eq, C::T_U + 128 * slot + 64 * ewg + 32), r1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            u[k] = __uint_as_float(r0[k]);
-            u[32 + k] = __uint_as_float(r1[k]);
-          }
+        const int bw = min(128, m - 128 * jb);
+        for (int ks = 0; ks < bw / 16; ++ks) {  // 16 features per step, two per TMEM column
+          const int fk = 128 * jb + 16 * ks;
+          const uint64_t bd =
+              sdesc_sw128(sbase + C::S_SP + (fk >> 6) * (C::NR * 128) + 32 * ((fk & 63) >> 4), 16, 1024);
+          mma_ts(tbase + C::T_O, tbase + C::T_U + 128 * sb + 8 * ks, bd, id2, (jb > 0 || ks > 0) ? 1u : 0u);
         }
-        const int fb = 128 * j + 64 * ewg;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          if (fb + k >= m) u[k] = -INFINITY;
-          mx = fmaxf(mx, u[k]);
+        mma_commit(bar(C::B_M2 + sb));
+        if (jb == nb - 1) {
+          mma_commit(bar(C::B_OF));
+          if (tb == n - 1 || kvh_of(T0 + tb + 1) - kvh0 != k) mma_commit(bar(C::B_SE));  // image released
         }
-        rmx[(g & 1) * 256 + ewg * 128 + r] = mx;
-        named_bar_sync(kBarEpi, kEpiThreads);
-        const float M = fmaxf(mx, rmx[(g & 1) * 256 + (1 - ewg) * 128 + r]);
-        bool need = false;
-        if (j == 0) {
-          c = M;
-        } else if (M > c + kTau) {
-          need = true;
-        }
-        if (__any_sync(0xffffffffu, need)) {  // raise this row's stabiliser: rescale O so far
-          mbar_wait(bar(C::B_SLOT + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, err);
-          tc_fence_after();
-          const float sc = need ? ex2(c - M) : 1.f;
-#pragma unroll
-          for (int cc = 0; cc < C::NR / 16; ++cc) {
-            const int col = C::T_O + ob * C::NR + ewg * (C::NR / 2) + 8 * cc;
-            uint32_t v[8];
-            tmem_ld8(taddr(tbase, eq, col), v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * sc);
-            tmem_st8(taddr(tbase, eq, col), v);
-          }
-          tmem_wait_st();
-          if (need) c = M;
-        }
-        {  // phi in fp32, written back over the same columns this thread read
-          uint32_t w0[32], w1[32];
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            w0[k] = __float_as_uint(ex2(u[k] - c));
-            w1[k] = __float_as_uint(ex2(u[32 + k] - c));
-          }
-          tmem_st32(taddr(tbase, eq, C::T_U + 128 * slot + 64 * ewg), w0);
-          tmem_st32(taddr(tbase, eq, C::T_U + 128 * slot + 64 * ewg + 32), w1);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::B_PHI + slot));
       }
-      // ---- output tile: out = O[:, :d] / O[:, d] ----
-      mbar_wait(bar(C::B_OF + ob), (it >> 1) & 1, abort_flag, err);
+      if (nblk >= 1)
+        mbar_wait(bar(C::B_M2 + (nblk - 1) % C::NU), ((nblk - 1) / C::NU) & 1, abort_flag, err, 200000000ull);
+    }
+  } else if (warp >= 4) {
+    // ---------------- epilogue warpgroup ----------------
+    const int eq = warp & 3;
+    const int r = eq * 32 + lane;  // query row within the tile (TMEM lane)
+    const bool issuer = (eq == 0 && lane == 0);
+    float v[128];  // the current block of this row: U + e
+    float c = 0.f;
+    const float4* ev = reinterpret_cast<const float4*>(smem + C::S_SP + C::NR * 128 * ((m + 63) / 64));
+    int pend = -1;  // tile whose output is waiting to be written
+    auto write_out = [&](int t) {  // out = O[:, :d] / O[:, d] -> bf16 -> staging -> TMA store
+      mbar_wait(bar(C::B_OF), t & 1, abort_flag, err);
       tc_fence_after();
-      uint32_t num[D / 2];
       uint32_t den;
+      tmem_ld1(taddr(tbase, eq, C::T_O + D), den);
+      tmem_wait_ld();
+      const float inv = 1.f / __uint_as_float(den);
+      if (issuer) bulk_wait_read<0>();  // the previous store has finished reading the staging tile
+      named_bar_sync(1, 128);
 #pragma unroll
-      for (int h2 = 0; h2 < D / 64; ++h2) {
+      for (int h2 = 0; h2 < D / 32; ++h2) {
         uint32_t t32[32];
-        tmem_ld32(taddr(tbase, eq, C::T_O + ob * C::NR + (D / 2) * ewg + 32 * h2), t32);
+        tmem_ld32(taddr(tbase, eq, C::T_O + 32 * h2), t32);
         tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 32; ++k) num[32 * h2 + k] = t32[k];
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            w4[k] = pack_bf16x2(__uint_as_float(t32[8 * c4 + 2 * k]) * inv,
+                                __uint_as_float(t32[8 * c4 + 2 * k + 1]) * inv);
+          const int cc = 4 * h2 + c4, rg = cc >> 3, c8 = cc & 7;
+          *reinterpret_cast<uint4*>(smem + C::S_OUT + rg * (128 * 128) + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
       }
-      tmem_ld1(taddr(tbase, eq, C::T_O + ob * C::NR + D), den);
-      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_OE + ob));
-      const float inv = 1.f / __uint_as_float(den);
-      const int T = T0 + it, bh = T / ntq, qt = T % ntq;
-      const int sb = it & 1;
-      if (issuer) bulk_wait_read<1>();
-      named_bar_sync(kBarStore, kEpiThreads);
-      // staging tile: 128 rows x D bf16, 64-dim regions of 128-byte rows, 128B swizzle
-#pragma unroll
-      for (int cc = 0; cc < D / 16; ++cc) {  // this thread's D/2 columns = D/16 chunks of 8
-        uint32_t w4[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          w4[k] = pack_bf16x2(__uint_as_float(num[8 * cc + 2 * k]) * inv, __uint_as_float(num[8 * cc + 2 * k + 1]) * inv);
-        const int chunk = (D / 16) * ewg + cc;  // 16-byte chunk index within the D-wide row
-        const int rg = chunk >> 3, c8 = chunk & 7;
-        *reinterpret_cast<uint4*>(smem + C::S_OUT + sb * C::QTILE + rg * (128 * 128) + r * 128 + ((c8 ^ (r & 7)) << 4)) =
-            make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
+      if (lane == 0) mbar_arrive(bar(C::B_OE));
       fence_proxy_async_smem();
-      named_bar_sync(kBarStore, kEpiThreads);
+      named_bar_sync(1, 128);
       if (issuer) {
+        const int T = T0 + t, bh = T / ntq, qt = T % ntq;
 #pragma unroll
         for (int rg = 0; rg < D / 64; ++rg)
-          tma_store_3d(&tmO, sbase + C::S_OUT + sb * C::QTILE + rg * (128 * 128), 64 * rg, qt * 128, bh);
+          tma_store_3d(&tmO, sbase + C::S_OUT + rg * (128 * 128), 64 * rg, qt * 128, bh);
         bulk_commit();
       }
+    };
+    if (nblk > 0) {  // block 0 in (its image is in shared memory once the first MMA2 could run)
+      mbar_wait(bar(C::B_UF + 0), 0, abort_flag, err);
+      mbar_wait(bar(C::B_SF), 0, abort_flag, err);
+      tc_fence_after();
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t t32[32];
+        tmem_ld32(taddr(tbase, eq, C::T_U + 32 * q4), t32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 e4 = ev[8 * q4 + k4];
+          v[32 * q4 + 4 * k4 + 0] = __uint_as_float(t32[4 * k4 + 0]) + e4.x;
+          v[32 * q4 + 4 * k4 + 1] = __uint_as_float(t32[4 * k4 + 1]) + e4.y;
+          v[32 * q4 + 4 * k4 + 2] = __uint_as_float(t32[4 * k4 + 2]) + e4.z;
+          v[32 * q4 + 4 * k4 + 3] = __uint_as_float(t32[4 * k4 + 3]) + e4.w;
+        }
+      }
     }
+    for (int g = 0; g < nblk; ++g) {
+      const int t = g / nb, j = g % nb, sg = g % C::NU;
+      const int fb = 128 * j;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 128; k += 2) {
+        if (fb + k >= m) v[k] = -INFINITY;
+        if (fb + k + 1 >= m) v[k + 1] = -INFINITY;
+        mx = max3(mx, v[k], v[k + 1]);
+      }
+      const bool need = (j > 0) && (mx > c + kTau);
+      if (j == 0) c = mx;
+      if (__any_sync(0xffffffffu, need)) {  // raise the stabiliser of the rows that need it
+        mbar_wait(bar(C::B_M2 + (g - 1) % C::NU), ((g - 1) / C::NU) & 1, abort_flag, err);
+        tc_fence_after();
+        scale_tmem_row(taddr(tbase, eq, C::T_O), C::NR / 8, need ? ex2(c - mx) : 1.f);
+      }
+      if (need) c = mx;
+      const bool more = g + 1 < nblk;
+      const int sn = (g + 1) % C::NU;
+      const int jn = (g + 1) % nb;
+      // the next block's exponents: its kv head's image must be in shared memory
+      const bool new_img = more && jn == 0 && kvh_of(T0 + (g + 1) / nb) != kvh_of(T0 + t);
+      if (more) {
+        mbar_wait(bar(C::B_UF + sn), ((g + 1) / C::NU) & 1, abort_flag, err);
+        tc_fence_after();
+      }
+      const int en = 32 * jn;  // float4 index of the next block's first exponent
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t nx[32];
+        if (more) tmem_ld32(taddr(tbase, eq, C::T_U + 128 * sn + 32 * q4), nx);  // next block streams in
+        uint32_t ph[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) ph[k] = pack_f16x2(ex2(v[32 * q4 + 2 * k] - c), ex2(v[32 * q4 + 2 * k + 1] - c));
+        tmem_st16(taddr(tbase, eq, C::T_U + 128 * sg + 16 * q4), ph);  // phi' over the U it came from
+        if (more) {
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[32 * q4 + k] = __uint_as_float(nx[k]);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_PHI + sg));
+      if (more) {  // the next block's exponents, once this block has been handed over (at a kv-head
+                   // change its image replaces this one only after this block's MMA2)
+        if (new_img) mbar_wait(bar(C::B_SF), (kvh_of(T0 + (g + 1) / nb) - kvh0) & 1, abort_flag, err);
+#pragma unroll
+        for (int k4 = 0; k4 < 32; ++k4) {
+          const float4 e4 = ev[en + k4];
+          v[4 * k4 + 0] += e4.x;
+          v[4 * k4 + 1] += e4.y;
+          v[4 * k4 + 2] += e4.z;
+          v[4 * k4 + 3] += e4.w;
+        }
+      }
+      // a finished tile's output is written after the next block has been handed to the MMA
+      // warp, so that the tensor core never waits for the readout
+      if (pend >= 0) {
+        write_out(pend);
+        pend = -1;
+      }
+      if (j == nb - 1) pend = t;
+    }
+    if (pend >= 0) write_out(pend);
     if (issuer) bulk_wait<0>();
   }
   tc_fence_before();
@@ -759,18 +1087,18 @@ int num_sms() {
 
 template <int D>
 int launch_key(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st) {
-  using C = KeyCfg<D>;
   CUtensorMap mk, mv;
   const int heads = p.B * p.Hkv;
   int rc = make_map(&mk, K, D, p.L, heads);
   if (rc == FAVOR_OK) rc = make_map(&mv, V, D, p.L, heads);
   if (rc != FAVOR_OK) return rc;
-  auto kern = key_pass_sm100<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  auto kern = (D == 64) ? key_pass_pp_sm100 : key_pass_sm100<D>;
+  const int smem_bytes = (D == 64) ? KeyPP::SMEM : KeyCfg<D>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass attribute: %s", cudaGetErrorString(e));
   char* base = static_cast<char*>(partials);
   dim3 grid((p.m + 127) / 128, p.P, heads);
-  kern<<<grid, kThreads, C::SMEM, st>>>(mk, mv, W, reinterpret_cast<float*>(base + p.part_S_off),
+  kern<<<grid, kThreads, smem_bytes, st>>>(mk, mv, W, reinterpret_cast<float*>(base + p.part_S_off),
                                         reinterpret_cast<float*>(base + p.part_c_off), p.L, p.m, p.P, p.chunk,
                                         p.nsb, p.wscale, p.nscale);
   e = cudaGetLastError();
@@ -792,7 +1120,7 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   const int ntiles = bh * ((p.L + 127) / 128);
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
   const unsigned char* img = static_cast<const unsigned char*>(state) + p.st_op_off;
-  kern<<<grid, kThreads, C::SMEM, st>>>(mq, mo, W, img, p.L, p.m, p.H, p.Hkv, ntiles, static_cast<int>(p.op_bytes),
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mo, W, img, p.L, p.m, p.H, p.Hkv, ntiles, static_cast<int>(p.op_bytes),
                                         p.wscale);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass launch: %s", cudaGetErrorString(e));

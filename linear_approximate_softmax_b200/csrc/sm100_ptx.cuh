@@ -49,6 +49,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the same condition (mbarrier.test_wait never suspends the thread,
+// unlike try_wait): for a thread that polls several barriers in turn.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with parity `parity` to complete.  Gives up after
 // `limit_ns` of wall time, or at once when *abort is set; on giving up it sets
 // *abort and the global error word and returns false.  Every pipeline wait in
@@ -69,6 +83,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       }
     }
   }
+}
+
+// Bookkeeping for a thread that polls several barriers with mbar_test: after a pass
+// that made no progress, counts it, and every 1024 such passes checks the SM clock;
+// gives up (setting *abort and the error word) after about 2^32 cycles (2-3 s) without
+// progress.  Reading a clock on every pass would cost more than the pass itself.
+__device__ __forceinline__ bool idle_poll(bool progressed, uint32_t& polls, long long& idle_since,
+                                          volatile int* abort, unsigned int* err_word) {
+  if (progressed) {
+    polls = 0;
+    return false;
+  }
+  if (polls == 0) idle_since = clock64();
+  if ((++polls & 1023u) == 0) {
+    if (*abort) return true;
+    if (clock64() - idle_since > (1ll << 32)) {
+      *abort = 1;
+      atomicOr(err_word, FAVOR_DEVERR_TIMEOUT);
+      return true;
+    }
+  }
+  return false;
 }
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
@@ -181,6 +217,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor of kind::f16 with fp16 A and B and an fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)                                   // D format: f32
+         | (0u << 7)                                 // A format: f16
+         | (0u << 10)                                // B format: f16
+         | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16)
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Instruction descriptor of kind::tf32 (fp32 operands read as tf32) with an fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4)                                   // D format: f32
@@ -235,10 +281,32 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 }
 
 // ---- arithmetic helpers ------------------------------------------------------------
+// One 3-input max on sm_100.  Volatile so that it stays between the tensor-memory load
+// that feeds it and the next one: otherwise the compiler may sink a whole pass of maxima
+// below later loads and keep every loaded value live.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm volatile("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ float ex2(float x) {  // hardware 2^x (MUFU), flushes subnormal results
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// Packs two floats as f16x2 (round to nearest even): `lo` in bits 15..0, `hi` in bits 31..16.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 // Packs two floats as bf16x2 (round to nearest even): `lo` in bits 15..0, `hi` in bits 31..16.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
