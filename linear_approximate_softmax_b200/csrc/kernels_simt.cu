@@ -176,14 +176,14 @@ __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
 
   const int f = blockIdx.x * 32 + (threadIdx.x >> 3);  // feature row (< op_atoms * 64)
   const int g = threadIdx.x & 7;                       // this thread's columns: g, g + 8, ...
-  constexpr int kMaxCols = (128 + 16) / 8;             // op_rows <= 144
+  constexpr int kMaxCols = (128 + 16) / 8;             // max(op_rows, D1) <= 144
   float val[kMaxCols];
-  float amax = 0.f;
+  float amax = 0.f, den = 0.f;
 #pragma unroll
   for (int k = 0; k < kMaxCols; ++k) {
     const int n = g + 8 * k;
     float acc = 0.f;
-    if (n < op_rows && f < m && n < D1) {
+    if (f < m && n < D1) {
       const size_t idx = static_cast<size_t>(f) * D1 + n;
       for (int p = 0; p < P; ++p) {
         const float c = pc[p * nsb + f / kStabBlock];
@@ -193,7 +193,8 @@ __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
       S[static_cast<size_t>(head) * m * D1 + idx] = acc;
     }
     val[k] = acc;
-    amax = fmaxf(amax, fabsf(acc));
+    if (n < op_rows) amax = fmaxf(amax, fabsf(acc));
+    if (n == D1 - 1) den = acc;
   }
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
@@ -214,7 +215,10 @@ __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
       *reinterpret_cast<__half*>(img + off) = __float2half_rn(ldexpf(val[k], -ex));
     }
   }
-  if (g == 0) reinterpret_cast<float*>(img + static_cast<size_t>(op_rows) * 128 * op_atoms)[f] = static_cast<float>(ex);
+  // tail: the exponent of each feature, then its normaliser entry with the same scaling
+  float* tail = reinterpret_cast<float*>(img + static_cast<size_t>(op_rows) * 128 * op_atoms);
+  if (g == 0) tail[f] = static_cast<float>(ex);
+  if (((D1 - 1) & 7) == g) tail[64 * op_atoms + f] = ldexpf(den, -ex);
 }
 
 // grid (ceil(L/32), B*H), 256 threads.

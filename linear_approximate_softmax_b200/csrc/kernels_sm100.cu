@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
           const uint4* row = reinterpret_cast<const uint4*>(smem + C::S_K + s * C::TILE + r * C::RGN + t * 128);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const uint4 v = row[c];
+            const uint4 v = row[c ^ (t & 7)];  // lanes of a wavefront start on different banks
             const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -406,10 +406,14 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
 // accumulators are merged exactly: S = 2^(c0-c) S0 + 2^(c1-c) S1.
 struct KeyPP {
   static constexpr int D = 64;
+  // warp 0 TMA producer, warps 1-2 MMA issuers, warps 3-10 two epilogue warpgroups (each covers
+  // the four TMEM lane quarters once, as warp % 4)
+  static constexpr int THREADS = 352;
+  static constexpr int EPI0 = 3;
   static constexpr int NST = 4;
   static constexpr int TILE = 128 * 64 * 2;
   static constexpr int NS = D + 16;
-  static constexpr int T_WHI = 0, T_WLO = 32, T_D1 = 64, T_S = 64 + 256;  // S[w] at T_S + NS*w
+  static constexpr int T_W = 0, T_D1 = 32, T_S = 32 + 256;  // W' fp16 | U^T x2 | S[w] at T_S + NS*w
   static_assert(T_S + 2 * NS <= 512, "TMEM budget");
   static constexpr int S_K = 0;
   static constexpr int S_V = S_K + NST * TILE;
@@ -418,14 +422,15 @@ struct KeyPP {
   static constexpr int S_ONES = S_V + NST * TILE;  // 128 tokens x 64 columns, column 0 = 1
   static constexpr int S_NRM = S_ONES + TILE;
   static constexpr int S_CW = S_NRM + NST * 512;   // final stabilisers, [warpgroup][feature]
-  static constexpr int S_BAR = S_CW + 1024;
-  static constexpr int B_KVF = 0, B_KVE = 4, B_D1F = 8, B_PHI = 10, B_SDONE = 12, NBAR = 14;
+  static constexpr int S_RED = S_CW + 1024;        // tile exponent maxima, [warpgroup][warp]
+  static constexpr int S_BAR = S_RED + 64;
+  static constexpr int B_KVF = 0, B_KVE = 4, B_D1F = 8, B_PHI = 10, B_SDONE = 12, B_CVT = 14, NBAR = 16;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int SMEM = S_ABORT + 16 + 1024;
 };
 
-__global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
+__global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const float* __restrict__ W,
     float* __restrict__ part_S, float* __restrict__ part_c, int L, int m, int P, int chunk, int nsb, float wscale,
     float nscale) {
@@ -456,6 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
       mbar_init(bar(C::B_D1F + w), 1);
       mbar_init(bar(C::B_PHI + w), 4);
       mbar_init(bar(C::B_SDONE + w), 1);
+      mbar_init(bar(C::B_CVT + w), 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -466,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
     tmem_alloc(smem_u32(tptr_slot), 512);
     tmem_relinquish();
   }
-  for (int i = tid; i < C::TILE / 4; i += kThreads) {  // ones atom: row t, logical column 0 = 1.0
+  for (int i = tid; i < C::TILE / 4; i += C::THREADS) {  // ones atom: row t, logical column 0 = 1.0
     const int t = i / 32, word = i % 32;                  // 32 words per 128-byte row
     // logical chunk 0 of row t sits at physical chunk (t % 8) under the 128-byte swizzle
     reinterpret_cast<uint32_t*>(smem + C::S_ONES)[i] = (word == (t & 7) * 4) ? 0x00003F80u : 0u;
@@ -477,32 +483,26 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
   tc_fence_after();
   const uint32_t tbase = *tptr_slot;
 
-  const bool epi = warp >= kEpiWarp0;
+  const bool epi = warp >= C::EPI0;
   const int eq = warp & 3;
-  const int ewg = (warp - kEpiWarp0) >> 2;
+  const int ewg = (warp - C::EPI0) >> 2;
   const int frow = eq * 32 + lane;
   const bool fvalid = frow < gw;
 
-  if (epi) {  // W' hi (warpgroup 0) / lo (warpgroup 1) into TMEM, lane = feature
+  if (epi) {  // W' as fp16 into TMEM, lane = feature; warpgroup ewg writes columns 16 ewg .. 16 ewg + 15
     const int f = f0 + frow;
-    uint32_t words[32];
+    uint32_t words[16];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < 16; ++j) {
       float w0 = 0.f, w1 = 0.f;
       if (fvalid) {
-        const float2 v = *reinterpret_cast<const float2*>(W + static_cast<size_t>(f) * D + 2 * j);
+        const float2 v = *reinterpret_cast<const float2*>(W + static_cast<size_t>(f) * D + 32 * ewg + 2 * j);
         w0 = v.x * wscale;
         w1 = v.y * wscale;
       }
-      if (ewg == 0) {
-        words[j] = pack_bf16x2(w0, w1);
-      } else {
-        const float h0 = __bfloat162float(__float2bfloat16_rn(w0));
-        const float h1 = __bfloat162float(__float2bfloat16_rn(w1));
-        words[j] = pack_bf16x2(w0 - h0, w1 - h1);
-      }
+      words[j] = pack_f16x2(w0, w1);
     }
-    tmem_st32(taddr(tbase, eq, ewg == 0 ? C::T_WHI : C::T_WLO), words);
+    tmem_st16(taddr(tbase, eq, C::T_W + 16 * ewg), words);
     tmem_wait_st();
   }
   tc_fence_before();
@@ -533,25 +533,20 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
     // wait behind the other's in a shared issue loop.
     if (lane == 0) {
       const int w = warp - 1;
-      const uint32_t id1 = idesc_bf16(128, 128, false, false);
+      const uint32_t id1 = idesc_f16(128, 128, false, false);
       const uint32_t idv = idesc_bf16(128, C::NS, false, true);  // N = 80: V, then the ones column
       const uint32_t d1 = tbase + C::T_D1 + 128 * w;
       const uint32_t sw = tbase + C::T_S + C::NS * w;
       int cnt = 0;
       for (int i = w; i < ntiles; i += 2, ++cnt) {
         const int s = i % C::NST;
-        if (!mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err)) break;
+        if (!mbar_wait(bar(C::B_CVT + w), cnt & 1, abort_flag, err)) break;  // K tile landed and converted
         if (cnt >= 1 && !mbar_wait(bar(C::B_SDONE + w), (cnt - 1) & 1, abort_flag, err)) break;  // U^T buffer free
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {  // MMA1: U^T = W' K^T (hi, then lo)
+        for (int ks = 0; ks < D / 16; ++ks) {  // MMA1: U^T = W' (2^-k K)^T in fp16
           const uint64_t bk = sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * ks, 16, 1024);
-          mma_ts(d1, tbase + C::T_WHI + 8 * ks, bk, id1, ks > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t bk = sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * ks, 16, 1024);
-          mma_ts(d1, tbase + C::T_WLO + 8 * ks, bk, id1, 1u);
+          mma_ts(d1, tbase + C::T_W + 8 * ks, bk, id1, ks > 0 ? 1u : 0u);
         }
         mma_commit(bar(C::B_D1F + w));
         if (!mbar_wait(bar(C::B_PHI + w), cnt & 1, abort_flag, err)) break;
@@ -592,31 +587,58 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
     float c_run = floor_c, tmax = -INFINITY;
     const uint32_t d1col = C::T_D1 + 128 * ewg;
     const uint32_t scol = C::T_S + C::NS * ewg;
-    // n(k) = |k|^2 * nscale of tile i's key frow (this thread's token), +inf past the chunk end;
-    // the 16-byte chunks of a swizzled row are summed in any order
-    auto key_norms = [&](int i) {
+    // Prepares tile i for its projection, one key row (token frow) per thread: stores -n(k) =
+    // -|k|^2 * nscale (-inf past the chunk end) and rewrites the bf16 row in place as fp16 times
+    // 2^-k, with one k per tile that puts the tile's largest |k| in [2^14, 2^15), so that the
+    // fp16 operand neither overflows nor loses the small values; returns 2^k.  The 16-byte
+    // chunks of a swizzled row are converted in place and summed in any order; thread frow starts
+    // at chunk frow % 8, so the eight threads of a shared-memory wavefront hit different banks.
+    int* red = reinterpret_cast<int*>(smem + C::S_RED) + 4 * ewg;
+    auto prepare_tile = [&](int i) -> float {
       const int s = i % C::NST;
       mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err);
-      const uint4* row = reinterpret_cast<const uint4*>(smem + C::S_K + s * C::TILE + frow * 128);
+      uint4* row = reinterpret_cast<uint4*>(smem + C::S_K + s * C::TILE + frow * 128);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t emax = 0;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const uint4 v = row[c];
+        const uint4 v = row[c ^ (frow & 7)];
         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float lo = __uint_as_float(wv[k] << 16), hi = __uint_as_float(wv[k] & 0xFFFF0000u);
           acc[k] = fmaf(lo, lo, acc[k]);
           acc[k] = fmaf(hi, hi, acc[k]);
+          emax = max(emax, max(wv[k] & 0x7F80u, (wv[k] >> 16) & 0x7F80u));
         }
       }
       const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-      nrm[s * 128 + frow] = (t_begin + 128 * i + frow < t_end) ? sum * nscale : INFINITY;
-      named_bar_sync(1 + ewg, 128);  // the warpgroup's 128 norms are in shared memory
+      nrm[s * 128 + frow] = (t_begin + 128 * i + frow < t_end) ? -sum * nscale : -INFINITY;
+      emax = __reduce_max_sync(0xffffffffu, emax);
+      if (lane == 0) red[eq] = static_cast<int>(emax >> 7);
+      named_bar_sync(1 + ewg, 128);
+      const int e = max(max(red[0], red[1]), max(red[2], red[3]));  // biased exponent of the tile max
+      const int k = min(100, max(-100, e - 141));                     // 2^(e-127) * 2^-k in [2^14, 2^15)
+      const float down = __int_as_float((127 - k) << 23);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {  // read again rather than hold 32 registers across the barrier
+        const uint4 v = row[c ^ (frow & 7)];
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          o[q] = pack_f16x2(__uint_as_float(wv[q] << 16) * down, __uint_as_float(wv[q] & 0xFFFF0000u) * down);
+        row[c ^ (frow & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();  // the converted row is read by the tensor cores
+      named_bar_sync(1 + ewg, 128);
+      if (tid == C::EPI0 * 32 + 128 * ewg) mbar_arrive(bar(C::B_CVT + ewg));
+      return __int_as_float((127 + k) << 23);
     };
     int cnt = 0;
-    if (ewg < ntiles) key_norms(ewg);
+    float up_next = ewg < ntiles ? prepare_tile(ewg) : 1.f;
     for (int i = ewg; i < ntiles; i += 2, ++cnt) {
+      const float up = up_next;
       const int s = i % C::NST;
       mbar_wait(bar(C::B_D1F + ewg), cnt & 1, abort_flag, err);
       tc_fence_after();
@@ -637,10 +659,10 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
           const float4 n4 = nv[8 * q4 + k4];
-          const float a0 = __uint_as_float(cur[4 * k4 + 0]) - n4.x;
-          const float a1 = __uint_as_float(cur[4 * k4 + 1]) - n4.y;
-          const float a2 = __uint_as_float(cur[4 * k4 + 2]) - n4.z;
-          const float a3 = __uint_as_float(cur[4 * k4 + 3]) - n4.w;
+          const float a0 = fmaf(__uint_as_float(cur[4 * k4 + 0]), up, n4.x);
+          const float a1 = fmaf(__uint_as_float(cur[4 * k4 + 1]), up, n4.y);
+          const float a2 = fmaf(__uint_as_float(cur[4 * k4 + 2]), up, n4.z);
+          const float a3 = fmaf(__uint_as_float(cur[4 * k4 + 3]), up, n4.w);
           tmax = max3(tmax, a0, a1);
           tmax = max3(tmax, a2, a3);
           wph[2 * k4] = pack_bf16x2(ex2(a0 - cc_run), ex2(a1 - cc_run));
@@ -661,11 +683,11 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_PHI + ewg));
-      if (i + 2 < ntiles) key_norms(i + 2);  // while this tile's MMA2 and the next MMA1 run
+      if (i + 2 < ntiles) up_next = prepare_tile(i + 2);  // while this tile's MMA2 runs
     }
     // merge the two accumulators row by row and write this group's partial state
     cw[ewg * 128 + frow] = c_run;
-    named_bar_sync(3, kEpiThreads);
+    named_bar_sync(3, 256);
     const float c0 = cw[frow], c1 = cw[128 + frow];
     const bool has1 = cnt_of[1] > 0;
     const float cmax = has1 ? fmaxf(c0, c1) : c0;
@@ -703,33 +725,45 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_pp_sm100(
 // ============================================================================
 template <int D>
 struct QueryCfg {
-  static constexpr int THREADS = 256;  // producer, MMA, two idle warps, one epilogue warpgroup (warps 4-7)
+  // warp 0 TMA producer, warps 1-2 MMA issuers (one per warpgroup), warp 3 idle,
+  // warps 4-11 two epilogue warpgroups on alternate tiles
+  static constexpr int THREADS = 384;
+  static constexpr int EPI0 = 4;
+  // d = 64: the normaliser comes out of MMA2 as a ones column (N = d + 16); d = 128: two
+  // accumulators of d + 16 columns do not fit in tensor memory next to two U buffers, so
+  // MMA2 has N = d and the epilogue sums phi' s_f for the normaliser
+  static constexpr bool DEN_MMA = D == 64;
+  static constexpr int NO = DEN_MMA ? D + 16 : D;  // MMA2 N = rows of the state image
+  static constexpr int MMAX = D == 64 ? 512 : 256;  // features held in shared memory
   static constexpr int QTILE = 128 * D * 2;
-  static constexpr int NR = D + 16;                  // output columns of MMA2 (values, normaliser, zeros)
-  static constexpr int MMAX = 256;                   // features held in shared memory
-  static constexpr int SP = NR * 128 * (MMAX / 64) + 4 * MMAX;  // fp16 state image + exponents (one buffer)
-  static constexpr int NU = 3;                       // U buffers: MMA1 runs up to two blocks ahead
-  // TMEM columns
-  static constexpr int T_U = 0;          // NU x 128
-  static constexpr int T_O = NU * 128;   // NR
-  static_assert(T_O + NR <= 512, "TMEM budget");
+  static constexpr int SP = NO * 128 * (MMAX / 64) + 8 * MMAX;  // fp16 image, exponents, fp32 normaliser column
+  // TMEM columns: warpgroup w owns U at w * TSTRIDE and O right after it
+  static constexpr int TSTRIDE = 128 + NO;
+  static_assert(2 * TSTRIDE <= 512, "TMEM budget");
   // shared memory
-  static constexpr int S_WHI = 0;
-  static constexpr int S_WLO = S_WHI + MMAX * 128 * (D / 64);
-  static constexpr int S_SP = S_WLO + MMAX * 128 * (D / 64);
-  static constexpr int S_Q = S_SP + SP;               // 2 stages, by tile parity
-  static constexpr int S_OUT = S_Q + 2 * QTILE;       // output staging
-  static constexpr int S_BAR = S_OUT + QTILE;
-  static constexpr int B_QF = 0, B_QE = 2, B_UF = 4, B_PHI = 7, B_M2 = 10, B_OF = 13, B_OE = 14, B_SF = 15,
-                       B_SE = 16, NBAR = 17;
+  static constexpr int S_W = 0;                          // W' fp16, [D/64 regions][MMAX rows][128 B]
+  static constexpr int S_SP = S_W + MMAX * 128 * (D / 64);
+  static constexpr int S_Q = S_SP + SP;                  // Q stage w belongs to warpgroup w
+  static constexpr int S_STG = S_Q + 2 * QTILE;          // output staging, one 64-column region, shared
+  static constexpr int S_BAR = S_STG + 128 * 128;
+  static constexpr int B_QF = 0, B_QE = 2, B_CVT = 4, B_UF = 6, B_PHI = 8, B_M2 = 10, B_OF = 12, B_OE = 14,
+                       B_SF = 16, B_SE = 17, B_STG = 18, NBAR = 19;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int SMEM = S_ABORT + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(S_SP % 1024 == 0 && S_Q % 1024 == 0 && S_STG % 1024 == 0 && (NO * 128) % 1024 == 0,
+                "128-byte swizzled operands start on 1024-byte boundaries");
 };
 
-// Query pass: one epilogue warpgroup; each thread owns one query row and holds a whole
-// 128-feature block of it in registers, so every U value is read from tensor memory once
-// and the row max is exact.  While it exponentiates block g it streams block g+1 in.
+// Query pass.  The CTA's tiles go alternately to two epilogue warpgroups, each with its own
+// U buffer, O accumulator, Q stage and MMA-issuing thread, so one warpgroup's exponentials
+// overlap the other's tensor-memory reads, waits and output.  Per 128-feature block a
+// warpgroup reads U twice from tensor memory: once for the exact row max of 2^k U + e, once
+// to exponentiate; the row stabiliser is raised lazily across blocks with an exact rescale
+// of O.  The projection runs in fp16: each warpgroup rewrites its next Q tile in place as
+// fp16 times 2^-k, one k per row that puts the row's largest |q| in [2^14, 2^15), and
+// multiplies that row's U by 2^k.
 template <int D>
 __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, const float* __restrict__ W,
@@ -749,32 +783,33 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   const int per = ntiles_total / gridDim.x, extra = ntiles_total % gridDim.x;
   const int T0 = blockIdx.x * per + min(static_cast<int>(blockIdx.x), extra);
   const int n = per + (static_cast<int>(blockIdx.x) < extra ? 1 : 0);
-  const int nblk = n * nb;  // blocks of this CTA, tile-major
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
   uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
   auto bar = [&](int i) { return sbase + C::S_BAR + 8u * i; };
   // kv head of a tile; non-decreasing along the tile order, so the CTA's tiles visit each
-  // kv head once and the image index of local tile it is kvh_of(T0 + it) - kvh_of(T0)
+  // kv head once: image index of local tile t = img(t), 0 .. nimg - 1
   auto kvh_of = [&](int T) {
     const int bh = T / ntq;
     return (bh / H) * Hkv + (bh % H) / G;
   };
   const int kvh0 = kvh_of(T0);
+  auto img = [&](int t) { return kvh_of(T0 + t) - kvh0; };
+  const int nimg = n > 0 ? img(n - 1) + 1 : 0;
 
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(C::B_QF + i), 1);
       mbar_init(bar(C::B_QE + i), 1);
-    }
-    for (int i = 0; i < C::NU; ++i) {
+      mbar_init(bar(C::B_CVT + i), 1);
       mbar_init(bar(C::B_UF + i), 1);
       mbar_init(bar(C::B_PHI + i), 4);
       mbar_init(bar(C::B_M2 + i), 1);
+      mbar_init(bar(C::B_OF + i), 1);
+      mbar_init(bar(C::B_OE + i), 4);
     }
-    mbar_init(bar(C::B_OF), 1);
-    mbar_init(bar(C::B_OE), 4);
     mbar_init(bar(C::B_SF), 1);
-    mbar_init(bar(C::B_SE), 1);
+    mbar_init(bar(C::B_SE), 2);  // an image is released once both issuers are done with it
+    mbar_init(bar(C::B_STG), 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmQ);
@@ -784,14 +819,14 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     tmem_alloc(smem_u32(tptr_slot), 512);
     tmem_relinquish();
   }
-  // W' = hi + lo as the K-major, 128B-swizzled B operand of MMA1: row f, 16-byte chunk c at c ^ (f % 8)
+  // W' in fp16 as the K-major, 128B-swizzled B operand of MMA1: row f, 16-byte chunk c at c ^ (f % 8)
   {
     const int rows = nb * 128;
     constexpr int CPR = D / 8;  // 16-byte chunks per row
     for (int item = tid; item < rows * CPR; item += NT) {
       const int f = item / CPR, c = item % CPR;
       const int rg = c >> 3, cc = c & 7;  // 64-dim region, chunk within the 128-byte row
-      uint32_t hi[4], lo[4];
+      uint32_t h[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         float w0 = 0.f, w1 = 0.f;
@@ -800,13 +835,10 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
           w0 = v.x * wscale;
           w1 = v.y * wscale;
         }
-        hi[k] = pack_bf16x2(w0, w1);
-        const float h0 = __uint_as_float(hi[k] << 16), h1 = __uint_as_float(hi[k] & 0xFFFF0000u);
-        lo[k] = pack_bf16x2(w0 - h0, w1 - h1);
+        h[k] = pack_f16x2(w0, w1);
       }
       const int off = rg * (C::MMAX * 128) + f * 128 + ((cc ^ (f & 7)) << 4);
-      *reinterpret_cast<uint4*>(smem + C::S_WHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(smem + C::S_WLO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(smem + C::S_W + off) = make_uint4(h[0], h[1], h[2], h[3]);
     }
   }
   fence_proxy_async_smem();
@@ -817,12 +849,11 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   unsigned int* err = &g_sm100_error_word;
 
   if (warp == 0) {
-    // ---------------- producer: Q tiles (2 stages) and state images ----------------
+    // ---------------- producer: Q tiles (stage = tile parity) and state images ----------------
     if (lane == 0) {
       int loaded = -1, issued = 0;
       for (int it = 0; it < n; ++it) {
         const int T = T0 + it, s = it & 1;
-        // the Q tile first: the previous image is released only after this tile's MMA1s
         if (it >= 2 && !mbar_wait(bar(C::B_QE + s), ((it >> 1) - 1) & 1, abort_flag, err)) break;
         mbar_arrive_expect_tx(bar(C::B_QF + s), C::QTILE);
         const int bh = T / ntq, qt = T % ntq;
@@ -830,8 +861,8 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         for (int r = 0; r < D / 64; ++r)
           tma_load_3d(sbase + C::S_Q + s * C::QTILE + r * (128 * 128), &tmQ, bar(C::B_QF + s), 64 * r, qt * 128, bh);
         issued = it + 1;
-        const int k = kvh_of(T) - kvh0;
-        if (k > loaded) {  // a new kv head: load its image once the previous one is released
+        const int k = img(it);
+        if (k > loaded) {  // a new kv head: load its image once both issuers have released the previous one
           if (k >= 1 && !mbar_wait(bar(C::B_SE), (k - 1) & 1, abort_flag, err)) break;
           mbar_arrive_expect_tx(bar(C::B_SF), op_bytes);
           bulk_load(sbase + C::S_SP, op_img + static_cast<size_t>(kvh0 + k) * op_bytes, op_bytes, bar(C::B_SF));
@@ -842,198 +873,262 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         mbar_wait(bar(C::B_QF + (it & 1)), (it >> 1) & 1, abort_flag, err, 200000000ull);
       if (loaded >= 0) mbar_wait(bar(C::B_SF), loaded & 1, abort_flag, err, 200000000ull);
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer: MMA1 up to two blocks ahead of MMA2 ----------------
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuer of warpgroup w = warp - 1: its tiles w, w + 2, ... ----------------
     if (lane == 0) {
-      const uint32_t id2 = idesc_f16(128, C::NR, false, false);
-      int a = 0;  // next block for MMA1
+      const int w = warp - 1;
+      const uint32_t id2 = idesc_f16(128, C::NO, false, false);
+      const uint32_t dU = tbase + w * C::TSTRIDE, dO = dU + 128;
+      const uint32_t qbase = sbase + C::S_Q + w * C::QTILE;
+      int cntb = 0, tc = 0, rel = 0;  // my blocks and tiles so far; images below rel released by me
       bool ok = true;
-      for (int b = 0; b < nblk && ok; ++b) {  // MMA2 of block b
-        while (a < nblk && a < b + C::NU) {
-          const int ta = a / nb, ja = a % nb, sa = a % C::NU;
-          if (ja == 0 && !mbar_wait(bar(C::B_QF + (ta & 1)), (ta >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          if (a >= C::NU && !mbar_wait(bar(C::B_M2 + sa), ((a / C::NU) - 1) & 1, abort_flag, err)) { ok = false; break; }
+      // releases image rel without having used it (after its predecessor's release completed,
+      // so that the arrival counts towards the right phase)
+      auto release_unused = [&]() {
+        if (rel >= 1 && !mbar_wait(bar(C::B_SE), (rel - 1) & 1, abort_flag, err)) return false;
+        mbar_arrive(bar(C::B_SE));
+        ++rel;
+        return true;
+      };
+      for (int t = w; t < n && ok; t += 2, ++tc) {
+        const int k = img(t);
+        while (rel < k && ok) ok = release_unused();
+        for (int j = 0; j < nb && ok; ++j, ++cntb) {
+          if (j == 0 && !mbar_wait(bar(C::B_CVT + w), tc & 1, abort_flag, err)) { ok = false; break; }
+          if (cntb >= 1 && !mbar_wait(bar(C::B_M2 + w), (cntb - 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          const int bw = min(128, m - 128 * ja);
-          const uint32_t id1 = idesc_bf16(128, bw, false, false);
-          const uint32_t dU = tbase + C::T_U + 128 * sa;
-          const uint32_t qbase = sbase + C::S_Q + (ta & 1) * C::QTILE;
+          const int bw = min(128, m - 128 * j);
+          const uint32_t id1 = idesc_f16(128, bw, false, false);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
+          for (int ks = 0; ks < D / 16; ++ks) {  // MMA1: U = (2^-k Q) W'^T in fp16
             const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
-            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * ja) * 128 + 32 * (ks & 3);
-            mma_ss(dU, sdesc_sw128(qbase + qo, 16, 1024), sdesc_sw128(sbase + C::S_WHI + wo, 16, 1024), id1,
+            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * j) * 128 + 32 * (ks & 3);
+            mma_ss(dU, sdesc_sw128(qbase + qo, 16, 1024), sdesc_sw128(sbase + C::S_W + wo, 16, 1024), id1,
                    ks > 0 ? 1u : 0u);
           }
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
-            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * ja) * 128 + 32 * (ks & 3);
-            mma_ss(dU, sdesc_sw128(qbase + qo, 16, 1024), sdesc_sw128(sbase + C::S_WLO + wo, 16, 1024), id1, 1u);
+          mma_commit(bar(C::B_UF + w));
+          if (j == nb - 1) mma_commit(bar(C::B_QE + w));  // the Q stage may take tile t + 2
+          if (!mbar_wait(bar(C::B_PHI + w), cntb & 1, abort_flag, err)) { ok = false; break; }
+          if (j == 0) {
+            if (tc >= 1 && !mbar_wait(bar(C::B_OE + w), (tc - 1) & 1, abort_flag, err)) { ok = false; break; }
+            if (!mbar_wait(bar(C::B_SF), k & 1, abort_flag, err)) { ok = false; break; }
           }
-          mma_commit(bar(C::B_UF + sa));
-          if (ja == nb - 1) mma_commit(bar(C::B_QE + (ta & 1)));
-          ++a;
-        }
-        if (!ok) break;
-        const int tb = b / nb, jb = b % nb, sb = b % C::NU;
-        if (!mbar_wait(bar(C::B_PHI + sb), (b / C::NU) & 1, abort_flag, err)) break;
-        const int k = kvh_of(T0 + tb) - kvh0;
-        if (jb == 0) {
-          if (tb >= 1 && !mbar_wait(bar(C::B_OE), (tb - 1) & 1, abort_flag, err)) break;
-          if (!mbar_wait(bar(C::B_SF), k & 1, abort_flag, err)) break;
-        }
-        tc_fence_after();
-        const int bw = min(128, m - 128 * jb);
-        for (int ks = 0; ks < bw / 16; ++ks) {  // 16 features per step, two per TMEM column
-          const int fk = 128 * jb + 16 * ks;
-          const uint64_t bd =
-              sdesc_sw128(sbase + C::S_SP + (fk >> 6) * (C::NR * 128) + 32 * ((fk & 63) >> 4), 16, 1024);
-          mma_ts(tbase + C::T_O, tbase + C::T_U + 128 * sb + 8 * ks, bd, id2, (jb > 0 || ks > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(C::B_M2 + sb));
-        if (jb == nb - 1) {
-          mma_commit(bar(C::B_OF));
-          if (tb == n - 1 || kvh_of(T0 + tb + 1) - kvh0 != k) mma_commit(bar(C::B_SE));  // image released
+          tc_fence_after();
+          for (int ks = 0; ks < bw / 16; ++ks) {  // MMA2: O += phi' S', 16 features per step, two per TMEM column
+            const int fk = 128 * j + 16 * ks;
+            const uint64_t bd =
+                sdesc_sw128(sbase + C::S_SP + (fk >> 6) * (C::NO * 128) + 32 * ((fk & 63) >> 4), 16, 1024);
+            mma_ts(dO, dU + 8 * ks, bd, id2, (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(C::B_M2 + w));
+          if (j == nb - 1) {
+            mma_commit(bar(C::B_OF + w));
+            const int knext = t + 2 < n ? img(t + 2) : nimg;
+            if (knext > k && k < nimg - 1) {  // done with image k: released when these MMAs complete
+              mma_commit(bar(C::B_SE));
+              rel = k + 1;
+            }
+          }
         }
       }
-      if (nblk >= 1)
-        mbar_wait(bar(C::B_M2 + (nblk - 1) % C::NU), ((nblk - 1) / C::NU) & 1, abort_flag, err, 200000000ull);
+      while (ok && rel < nimg - 1) ok = release_unused();
+      if (cntb >= 1) mbar_wait(bar(C::B_M2 + w), (cntb - 1) & 1, abort_flag, err, 200000000ull);
     }
-  } else if (warp >= 4) {
-    // ---------------- epilogue warpgroup ----------------
+  } else if (warp >= C::EPI0) {
+    // ---------------- epilogue warpgroup ewg: tiles ewg, ewg + 2, ... ----------------
     const int eq = warp & 3;
+    const int ewg = (warp - C::EPI0) >> 2;
     const int r = eq * 32 + lane;  // query row within the tile (TMEM lane)
     const bool issuer = (eq == 0 && lane == 0);
-    float v[128];  // the current block of this row: U + e
-    float c = 0.f;
-    const float4* ev = reinterpret_cast<const float4*>(smem + C::S_SP + C::NR * 128 * ((m + 63) / 64));
-    int pend = -1;  // tile whose output is waiting to be written
-    auto write_out = [&](int t) {  // out = O[:, :d] / O[:, d] -> bf16 -> staging -> TMA store
-      mbar_wait(bar(C::B_OF), t & 1, abort_flag, err);
-      tc_fence_after();
-      uint32_t den;
-      tmem_ld1(taddr(tbase, eq, C::T_O + D), den);
-      tmem_wait_ld();
-      const float inv = 1.f / __uint_as_float(den);
-      if (issuer) bulk_wait_read<0>();  // the previous store has finished reading the staging tile
-      named_bar_sync(1, 128);
+    const uint32_t cU = ewg * C::TSTRIDE, cO = cU + 128;  // TMEM columns
+    const int atoms = (m + 63) / 64;  // the image holds [atoms][NO rows][64 features] fp16, then its tail
+    const float* ev = reinterpret_cast<const float*>(smem + C::S_SP + C::NO * 128 * atoms);
+    const float* sd = ev + 64 * atoms;  // fp32 normaliser column of the state, same scaling as the image
+    // rewrites row r of Q tile t (Q stage ewg) as fp16 x 2^-k; returns 2^k.  Thread r starts at
+    // chunk r % 8 so that the eight threads of a shared-memory wavefront hit different banks.
+    auto prepare = [&](int t, int tcount) -> float {
+      mbar_wait(bar(C::B_QF + ewg), tcount & 1, abort_flag, err);
+      unsigned char* qrow = smem + C::S_Q + ewg * C::QTILE + r * 128;
+      uint32_t emax = 0;
 #pragma unroll
-      for (int h2 = 0; h2 < D / 32; ++h2) {
-        uint32_t t32[32];
-        tmem_ld32(taddr(tbase, eq, C::T_O + 32 * h2), t32);
-        tmem_wait_ld();
+      for (int rg = 0; rg < D / 64; ++rg)
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t w4[4];
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(qrow + rg * (128 * 128) + 16 * (c ^ (r & 7)));
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            w4[k] = pack_bf16x2(__uint_as_float(t32[8 * c4 + 2 * k]) * inv,
-                                __uint_as_float(t32[8 * c4 + 2 * k + 1]) * inv);
-          const int cc = 4 * h2 + c4, rg = cc >> 3, c8 = cc & 7;
-          *reinterpret_cast<uint4*>(smem + C::S_OUT + rg * (128 * 128) + r * 128 + ((c8 ^ (r & 7)) << 4)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int k = 0; k < 4; ++k) emax = max(emax, max(wv[k] & 0x7F80u, (wv[k] >> 16) & 0x7F80u));
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_OE));
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (issuer) {
-        const int T = T0 + t, bh = T / ntq, qt = T % ntq;
+      const int k = min(100, max(-100, static_cast<int>(emax >> 7) - 141));
+      const float down = __int_as_float((127 - k) << 23);
 #pragma unroll
-        for (int rg = 0; rg < D / 64; ++rg)
-          tma_store_3d(&tmO, sbase + C::S_OUT + rg * (128 * 128), 64 * rg, qt * 128, bh);
-        bulk_commit();
-      }
+      for (int rg = 0; rg < D / 64; ++rg)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4* p = reinterpret_cast<uint4*>(qrow + rg * (128 * 128) + 16 * (c ^ (r & 7)));
+          const uint4 v = *p;
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            o[q] = pack_f16x2(__uint_as_float(wv[q] << 16) * down, __uint_as_float(wv[q] & 0xFFFF0000u) * down);
+          *p = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      fence_proxy_async_smem();  // the converted tile is read by the tensor cores
+      named_bar_sync(1 + ewg, 128);
+      if (issuer) mbar_arrive(bar(C::B_CVT + ewg));
+      return __int_as_float((127 + k) << 23);
     };
-    if (nblk > 0) {  // block 0 in (its image is in shared memory once the first MMA2 could run)
-      mbar_wait(bar(C::B_UF + 0), 0, abort_flag, err);
-      mbar_wait(bar(C::B_SF), 0, abort_flag, err);
-      tc_fence_after();
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t t32[32];
-        tmem_ld32(taddr(tbase, eq, C::T_U + 32 * q4), t32);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const float4 e4 = ev[8 * q4 + k4];
-          v[32 * q4 + 4 * k4 + 0] = __uint_as_float(t32[4 * k4 + 0]) + e4.x;
-          v[32 * q4 + 4 * k4 + 1] = __uint_as_float(t32[4 * k4 + 1]) + e4.y;
-          v[32 * q4 + 4 * k4 + 2] = __uint_as_float(t32[4 * k4 + 2]) + e4.z;
-          v[32 * q4 + 4 * k4 + 3] = __uint_as_float(t32[4 * k4 + 3]) + e4.w;
-        }
-      }
-    }
-    for (int g = 0; g < nblk; ++g) {
-      const int t = g / nb, j = g % nb, sg = g % C::NU;
-      const int fb = 128 * j;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < 128; k += 2) {
-        if (fb + k >= m) v[k] = -INFINITY;
-        if (fb + k + 1 >= m) v[k + 1] = -INFINITY;
-        mx = max3(mx, v[k], v[k + 1]);
-      }
-      const bool need = (j > 0) && (mx > c + kTau);
-      if (j == 0) c = mx;
-      if (__any_sync(0xffffffffu, need)) {  // raise the stabiliser of the rows that need it
-        mbar_wait(bar(C::B_M2 + (g - 1) % C::NU), ((g - 1) / C::NU) & 1, abort_flag, err);
+    float up_next = ewg < n ? prepare(ewg, 0) : 1.f;
+    int cntb = 0, tc = 0;
+    for (int t = ewg; t < n; t += 2, ++tc) {
+      const float up = up_next;
+      mbar_wait(bar(C::B_SF), img(t) & 1, abort_flag, err);  // this tile's image (exponents) is in
+      float c = 0.f, den = 0.f;
+      for (int j = 0; j < nb; ++j, ++cntb) {
+        mbar_wait(bar(C::B_UF + ewg), cntb & 1, abort_flag, err);
         tc_fence_after();
-        scale_tmem_row(taddr(tbase, eq, C::T_O), C::NR / 8, need ? ex2(c - mx) : 1.f);
-      }
-      if (need) c = mx;
-      const bool more = g + 1 < nblk;
-      const int sn = (g + 1) % C::NU;
-      const int jn = (g + 1) % nb;
-      // the next block's exponents: its kv head's image must be in shared memory
-      const bool new_img = more && jn == 0 && kvh_of(T0 + (g + 1) / nb) != kvh_of(T0 + t);
-      if (more) {
-        mbar_wait(bar(C::B_UF + sn), ((g + 1) / C::NU) & 1, abort_flag, err);
-        tc_fence_after();
-      }
-      const int en = 32 * jn;  // float4 index of the next block's first exponent
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t nx[32];
-        if (more) tmem_ld32(taddr(tbase, eq, C::T_U + 128 * sn + 32 * q4), nx);  // next block streams in
-        uint32_t ph[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) ph[k] = pack_f16x2(ex2(v[32 * q4 + 2 * k] - c), ex2(v[32 * q4 + 2 * k + 1] - c));
-        tmem_st16(taddr(tbase, eq, C::T_U + 128 * sg + 16 * q4), ph);  // phi' over the U it came from
-        if (more) {
+        const float4* e4p = reinterpret_cast<const float4*>(ev + 128 * j);
+        const bool ragged = 128 * j + 128 > m;  // features past m in this block (warp-uniform)
+        // pass 1: row max of 2^k U + e over the block
+        float mx;
+        {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          uint32_t cur[32], nxt[32];
+          tmem_ld32(taddr(tbase, eq, cU), cur);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) v[32 * q4 + k] = __uint_as_float(nx[k]);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_PHI + sg));
-      if (more) {  // the next block's exponents, once this block has been handed over (at a kv-head
-                   // change its image replaces this one only after this block's MMA2)
-        if (new_img) mbar_wait(bar(C::B_SF), (kvh_of(T0 + (g + 1) / nb) - kvh0) & 1, abort_flag, err);
+          for (int q4 = 0; q4 < 4; ++q4) {
+            if (q4 < 3) tmem_ld32(taddr(tbase, eq, cU + 32 * (q4 + 1)), nxt);
 #pragma unroll
-        for (int k4 = 0; k4 < 32; ++k4) {
-          const float4 e4 = ev[en + k4];
-          v[4 * k4 + 0] += e4.x;
-          v[4 * k4 + 1] += e4.y;
-          v[4 * k4 + 2] += e4.z;
-          v[4 * k4 + 3] += e4.w;
+            for (int k4 = 0; k4 < 8; ++k4) {
+              const float4 e4 = e4p[8 * q4 + k4];
+              float a[4] = {fmaf(__uint_as_float(cur[4 * k4 + 0]), up, e4.x),
+                            fmaf(__uint_as_float(cur[4 * k4 + 1]), up, e4.y),
+                            fmaf(__uint_as_float(cur[4 * k4 + 2]), up, e4.z),
+                            fmaf(__uint_as_float(cur[4 * k4 + 3]), up, e4.w)};
+              if (ragged) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (128 * j + 32 * q4 + 4 * k4 + e >= m) a[e] = -INFINITY;
+              }
+              m4[k4 & 3] = max3(m4[k4 & 3], a[0], a[1]);
+              m4[k4 & 3] = max3(m4[k4 & 3], a[2], a[3]);
+            }
+            if (q4 < 3) {
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) cur[k] = nxt[k];
+            }
+          }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        }
+        const bool need = (j > 0) && (mx > c + kTau);
+        if (j == 0) c = mx;
+        if (__any_sync(0xffffffffu, need)) {  // raise the stabiliser of the rows that need it
+          mbar_wait(bar(C::B_M2 + ewg), (cntb - 1) & 1, abort_flag, err);  // O holds the previous blocks
+          tc_fence_after();
+          const float f = need ? ex2(c - mx) : 1.f;
+          scale_tmem_row(taddr(tbase, eq, cO), C::NO / 8, f);
+          den *= f;
+        }
+        if (need) c = mx;
+        // pass 2: phi' = 2^(2^k U + e - c) as fp16 over the first 64 columns of U
+        {
+          uint32_t cur[32], nxt[32];
+          tmem_ld32(taddr(tbase, eq, cU), cur);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            if (q4 < 3) tmem_ld32(taddr(tbase, eq, cU + 32 * (q4 + 1)), nxt);
+            uint32_t ph[16];
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+              const float4 e4 = e4p[8 * q4 + k4];
+              float a[4] = {fmaf(__uint_as_float(cur[4 * k4 + 0]), up, e4.x),
+                            fmaf(__uint_as_float(cur[4 * k4 + 1]), up, e4.y),
+                            fmaf(__uint_as_float(cur[4 * k4 + 2]), up, e4.z),
+                            fmaf(__uint_as_float(cur[4 * k4 + 3]), up, e4.w)};
+              if (ragged) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (128 * j + 32 * q4 + 4 * k4 + e >= m) a[e] = -INFINITY;
+              }
+              const float p0 = ex2(a[0] - c), p1 = ex2(a[1] - c), p2 = ex2(a[2] - c), p3 = ex2(a[3] - c);
+              if constexpr (!C::DEN_MMA) {
+                const float4 s4 = reinterpret_cast<const float4*>(sd + 128 * j)[8 * q4 + k4];
+                den = fmaf(p0, s4.x, fmaf(p1, s4.y, fmaf(p2, s4.z, fmaf(p3, s4.w, den))));
+              }
+              ph[2 * k4] = pack_f16x2(p0, p1);
+              ph[2 * k4 + 1] = pack_f16x2(p2, p3);
+            }
+            tmem_st16(taddr(tbase, eq, cU + 16 * q4), ph);  // phi' over columns already read
+            if (q4 < 3) {
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) cur[k] = nxt[k];
+            }
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_PHI + ewg));
+      }
+      // the tile's blocks are handed over: convert the next tile's Q while the last MMA2 runs
+      if (t + 2 < n) up_next = prepare(t + 2, tc + 1);
+      // out = O[:, :d] / den -> bf16 -> shared staging (taken in tile order) -> TMA store
+      mbar_wait(bar(C::B_OF + ewg), tc & 1, abort_flag, err);
+      tc_fence_after();
+      if constexpr (C::DEN_MMA) {
+        uint32_t dv;
+        tmem_ld1(taddr(tbase, eq, cO + D), dv);
+        tmem_wait_ld();
+        den = __uint_as_float(dv);
+      }
+      const float inv = 1.f / den;
+      if (t >= 1) mbar_wait(bar(C::B_STG), (t - 1) & 1, abort_flag, err);  // tile t - 1 released the staging tile
+      const int T = T0 + t, bh = T / ntq, qt = T % ntq;
+#pragma unroll
+      for (int rg = 0; rg < D / 64; ++rg) {
+        if (rg > 0) {
+          if (issuer) bulk_wait_read<0>();  // the previous region's store has read the staging tile
+          named_bar_sync(1 + ewg, 128);
+        }
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t t32[32];
+          tmem_ld32(taddr(tbase, eq, cO + 64 * rg + 32 * h2), t32);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              w4[k] = pack_bf16x2(__uint_as_float(t32[8 * c4 + 2 * k]) * inv,
+                                  __uint_as_float(t32[8 * c4 + 2 * k + 1]) * inv);
+            const int c8 = 4 * h2 + c4;
+            *reinterpret_cast<uint4*>(smem + C::S_STG + r * 128 + ((c8 ^ (r & 7)) << 4)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+        if (rg == D / 64 - 1) {  // all of O has been read: the next tile may accumulate into it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::B_OE + ewg));
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1 + ewg, 128);
+        if (issuer) {
+          tma_store_3d(&tmO, sbase + C::S_STG, 64 * rg, qt * 128, bh);
+          bulk_commit();
         }
       }
-      // a finished tile's output is written after the next block has been handed to the MMA
-      // warp, so that the tensor core never waits for the readout
-      if (pend >= 0) {
-        write_out(pend);
-        pend = -1;
+      if (issuer) {
+        bulk_wait_read<0>();
+        mbar_arrive(bar(C::B_STG));  // the staging tile is free for tile t + 1
       }
-      if (j == nb - 1) pend = t;
     }
-    if (pend >= 0) write_out(pend);
     if (issuer) bulk_wait<0>();
   }
   tc_fence_before();
@@ -1094,11 +1189,12 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   if (rc != FAVOR_OK) return rc;
   auto kern = (D == 64) ? key_pass_pp_sm100 : key_pass_sm100<D>;
   const int smem_bytes = (D == 64) ? KeyPP::SMEM : KeyCfg<D>::SMEM;
+  const int threads = (D == 64) ? KeyPP::THREADS : kThreads;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass attribute: %s", cudaGetErrorString(e));
   char* base = static_cast<char*>(partials);
   dim3 grid((p.m + 127) / 128, p.P, heads);
-  kern<<<grid, kThreads, smem_bytes, st>>>(mk, mv, W, reinterpret_cast<float*>(base + p.part_S_off),
+  kern<<<grid, threads, smem_bytes, st>>>(mk, mv, W, reinterpret_cast<float*>(base + p.part_S_off),
                                         reinterpret_cast<float*>(base + p.part_c_off), p.L, p.m, p.P, p.chunk,
                                         p.nsb, p.wscale, p.nscale);
   e = cudaGetLastError();
@@ -1130,14 +1226,16 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
 }  // namespace
 
 bool sm100_key_supported(const Plan& p) { return p.d == 64 || p.d == 128; }
-bool sm100_query_supported(const Plan& p) { return p.d == 64 && p.m <= QueryCfg<64>::MMAX; }
+bool sm100_query_supported(const Plan& p) {
+  return (p.d == 64 && p.m <= QueryCfg<64>::MMAX) || (p.d == 128 && p.m <= QueryCfg<128>::MMAX);
+}
 
 int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st) {
   return p.d == 64 ? launch_key<64>(K, V, W, partials, p, st) : launch_key<128>(K, V, W, partials, p, st);
 }
 
 int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st) {
-  return launch_query<64>(Q, W, state, out, p, st);
+  return p.d == 64 ? launch_query<64>(Q, W, state, out, p, st) : launch_query<128>(Q, W, state, out, p, st);
 }
 
 int sm100_read_and_clear_error(unsigned int* word) {
