@@ -112,9 +112,8 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
   p->st_S_off = 0;
   p->st_c_off = round_up(sizeof(float) * heads * m * D1, 256);
   p->st_op_off = p->st_c_off + round_up(sizeof(float) * heads, 256);
-  // the query pass's state operand: d = 64 carries the normaliser as an extra row (padded to
-  // d + 16 rows for the MMA), d = 128 keeps d rows and reads the normaliser from the tail
-  p->op_rows = d == 64 ? d + 16 : d;
+  // the query pass's state operand: d rows of fp16 (the normaliser column goes to the tail)
+  p->op_rows = d;
   p->op_atoms = (m + 63) / 64;
   // fp16 rows (64 features per 128-byte row), then one fp32 exponent per feature, then the
   // fp32 normaliser column with the same per-feature scaling

@@ -55,6 +55,8 @@ constexpr int kEpiWarp0 = 4;
 constexpr int kEpiThreads = 256;
 constexpr uint32_t kBarEpi = 1;    // named barrier: epilogue max exchange (lock-step key pass)
 constexpr float kTau = 8.f;        // lazy stabiliser threshold (log2 units)
+// registers per thread after setmaxnreg: producer / MMA warpgroup, epilogue warpgroups
+constexpr int kRegsLow = 96, kRegsHigh = 200;
 
 __device__ __forceinline__ uint32_t taddr(uint32_t base, int lane_quarter, int col) {
   return base + (static_cast<uint32_t>(lane_quarter * 32) << 16) + static_cast<uint32_t>(col);
@@ -398,36 +400,37 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
 // ============================================================================
 // Key pass, d = 64: the two epilogue warpgroups take alternate tiles
 // ============================================================================
-// Each warpgroup owns one U^T buffer, one S accumulator, its own running
-// stabiliser and its own MMA-issuing thread (warp 1 for warpgroup 0, warp 2 for
-// warpgroup 1), so one warpgroup's exp work overlaps the other's TMEM loads and
-// MMAs.  A warpgroup computes the key norms of its next tile itself, between
-// handing phi to its MMA2 and the arrival of its next U^T.  At the end the two
-// accumulators are merged exactly: S = 2^(c0-c) S0 + 2^(c1-c) S1.
+// Each warpgroup owns a U^T buffer, a phi buffer and an S accumulator in tensor
+// memory, its own running stabilisers and its own MMA-issuing thread (warp 1 for
+// warpgroup 0, warp 2 for warpgroup 1).  The epilogue releases U^T as soon as it
+// has read it, so the next tile's projection runs while this tile's exponentials
+// and its contraction finish; phi goes to its own buffer.  A warpgroup prepares
+// (norms, fp16 conversion) the tile after its current one before waiting for the
+// current U^T.  The normaliser column sum_t phi is accumulated by the epilogue
+// itself, in fp32.  At the end the two accumulators are merged exactly:
+// S = 2^(c0-c) S0 + 2^(c1-c) S1.
 struct KeyPP {
   static constexpr int D = 64;
-  // warp 0 TMA producer, warps 1-2 MMA issuers, warps 3-10 two epilogue warpgroups (each covers
-  // the four TMEM lane quarters once, as warp % 4)
-  static constexpr int THREADS = 352;
-  static constexpr int EPI0 = 3;
-  static constexpr int NST = 4;
+  // warp 0 TMA producer, warps 1-2 MMA issuers, warp 3 idle, warps 4-11 two epilogue
+  // warpgroups (each covers the four TMEM lane quarters once, as warp % 4)
+  static constexpr int THREADS = 384;
+  static constexpr int EPI0 = 4;
+  static constexpr int NST = 6;  // K/V stages: a tile is prepared two tiles ahead of its use
   static constexpr int TILE = 128 * 64 * 2;
-  static constexpr int NS = D + 16;
-  static constexpr int T_W = 0, T_D1 = 32, T_S = 32 + 256;  // W' fp16 | U^T x2 | S[w] at T_S + NS*w
-  static_assert(T_S + 2 * NS <= 512, "TMEM budget");
-  static constexpr int S_K = 0;
+  // TMEM columns: warpgroup w owns U^T at 256 w, phi at 256 w + 128 (bf16 pairs), S at 256 w + 192
+  static constexpr int T_U = 0, T_P = 128, T_S = 192, T_STRIDE = 256;
+  static constexpr int S_W = 0;                     // W' fp16, 128 features x 64 dims, K-major SW128 (A of MMA1)
+  static constexpr int S_K = S_W + 128 * 128;
   static constexpr int S_V = S_K + NST * TILE;
-  // [V | 1] as one N = 80 MN-major operand: the ones column is the first column of a
-  // second 64-column atom, LBO bytes after the V tile of the stage
-  static constexpr int S_ONES = S_V + NST * TILE;  // 128 tokens x 64 columns, column 0 = 1
-  static constexpr int S_NRM = S_ONES + TILE;
-  static constexpr int S_CW = S_NRM + NST * 512;   // final stabilisers, [warpgroup][feature]
-  static constexpr int S_RED = S_CW + 1024;        // tile exponent maxima, [warpgroup][warp]
-  static constexpr int S_BAR = S_RED + 64;
-  static constexpr int B_KVF = 0, B_KVE = 4, B_D1F = 8, B_PHI = 10, B_SDONE = 12, B_CVT = 14, NBAR = 16;
+  static constexpr int S_NRM = S_V + NST * TILE;    // per stage: -n(k) [128], then 2^s [128]
+  static constexpr int S_CW = S_NRM + NST * 1024;   // final stabilisers and normalisers, [2][2][128]
+  static constexpr int S_BAR = S_CW + 2048;
+  static constexpr int B_KVF = 0, B_KVE = NST, B_CVT = 2 * NST, B_D1F = B_CVT + 2, B_UE = B_D1F + 2,
+                       B_PHI = B_UE + 2, B_SDONE = B_PHI + 2, NBAR = B_SDONE + 2;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int SMEM = S_ABORT + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
@@ -458,10 +461,11 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       mbar_init(bar(C::B_KVE + s), 1);
     }
     for (int w = 0; w < 2; ++w) {
+      mbar_init(bar(C::B_CVT + w), 1);
       mbar_init(bar(C::B_D1F + w), 1);
+      mbar_init(bar(C::B_UE + w), 4);
       mbar_init(bar(C::B_PHI + w), 4);
       mbar_init(bar(C::B_SDONE + w), 1);
-      mbar_init(bar(C::B_CVT + w), 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -472,45 +476,34 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     tmem_alloc(smem_u32(tptr_slot), 512);
     tmem_relinquish();
   }
-  for (int i = tid; i < C::TILE / 4; i += C::THREADS) {  // ones atom: row t, logical column 0 = 1.0
-    const int t = i / 32, word = i % 32;                  // 32 words per 128-byte row
-    // logical chunk 0 of row t sits at physical chunk (t % 8) under the 128-byte swizzle
-    reinterpret_cast<uint32_t*>(smem + C::S_ONES)[i] = (word == (t & 7) * 4) ? 0x00003F80u : 0u;
+  // W' fp16 as the K-major 128B-swizzled A operand of MMA1: row f, 16-byte chunk c at c ^ (f % 8)
+  for (int item = tid; item < 128 * 8; item += C::THREADS) {
+    const int f = item >> 3, c = item & 7;
+    uint32_t h[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float w0 = 0.f, w1 = 0.f;
+      if (f < gw) {
+        const float2 v = *reinterpret_cast<const float2*>(W + static_cast<size_t>(f0 + f) * D + 8 * c + 2 * k);
+        w0 = v.x * wscale;
+        w1 = v.y * wscale;
+      }
+      h[k] = pack_f16x2(w0, w1);
+    }
+    *reinterpret_cast<uint4*>(smem + C::S_W + f * 128 + ((c ^ (f & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tptr_slot;
-
-  const bool epi = warp >= C::EPI0;
-  const int eq = warp & 3;
-  const int ewg = (warp - C::EPI0) >> 2;
-  const int frow = eq * 32 + lane;
-  const bool fvalid = frow < gw;
-
-  if (epi) {  // W' as fp16 into TMEM, lane = feature; warpgroup ewg writes columns 16 ewg .. 16 ewg + 15
-    const int f = f0 + frow;
-    uint32_t words[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      float w0 = 0.f, w1 = 0.f;
-      if (fvalid) {
-        const float2 v = *reinterpret_cast<const float2*>(W + static_cast<size_t>(f) * D + 32 * ewg + 2 * j);
-        w0 = v.x * wscale;
-        w1 = v.y * wscale;
-      }
-      words[j] = pack_f16x2(w0, w1);
-    }
-    tmem_st16(taddr(tbase, eq, C::T_W + 16 * ewg), words);
-    tmem_wait_st();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-
   unsigned int* err = &g_sm100_error_word;
-  const int cnt_of[2] = {(ntiles + 1) / 2, ntiles / 2};  // tiles of each warpgroup
+
+  // registers: the producer / MMA warpgroup gives part of its share to the two epilogue
+  // warpgroups (128 x 96 + 256 x 200 = 63488 <= 384 x 168, the launch allocation; the host
+  // checks the compiled count before launching)
+  if (warp < C::EPI0) {
+  setmaxnreg_dec<kRegsLow>();
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
@@ -528,34 +521,43 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
         mbar_wait(bar(C::B_KVF + i % C::NST), (i / C::NST) & 1, abort_flag, err, 200000000ull);
     }
   } else if (warp == 1 || warp == 2) {
-    // ---------------- MMA issuers: warp 1 serves warpgroup 0, warp 2 warpgroup 1 ----------------
-    // One issuing thread per warpgroup, each in tile order, so neither warpgroup's MMAs
-    // wait behind the other's in a shared issue loop.
+    // ---------------- MMA issuer of warpgroup w: tiles w, w + 2, ... ----------------
+    // The next tile's projection is issued as soon as the epilogue has read this tile's
+    // U^T, ahead of this tile's contraction.
     if (lane == 0) {
       const int w = warp - 1;
       const uint32_t id1 = idesc_f16(128, 128, false, false);
-      const uint32_t idv = idesc_bf16(128, C::NS, false, true);  // N = 80: V, then the ones column
-      const uint32_t d1 = tbase + C::T_D1 + 128 * w;
-      const uint32_t sw = tbase + C::T_S + C::NS * w;
-      int cnt = 0;
-      for (int i = w; i < ntiles; i += 2, ++cnt) {
+      const uint32_t idv = idesc_bf16(128, D, false, true);  // V tile as an MN-major B operand
+      const uint32_t dU = tbase + w * C::T_STRIDE + C::T_U, dP = tbase + w * C::T_STRIDE + C::T_P,
+                     dS = tbase + w * C::T_STRIDE + C::T_S;
+      auto mma1 = [&](int i) {  // U^T = W' (2^-s K)^T in fp16
         const int s = i % C::NST;
-        if (!mbar_wait(bar(C::B_CVT + w), cnt & 1, abort_flag, err)) break;  // K tile landed and converted
-        if (cnt >= 1 && !mbar_wait(bar(C::B_SDONE + w), (cnt - 1) & 1, abort_flag, err)) break;  // U^T buffer free
-        tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {  // MMA1: U^T = W' (2^-k K)^T in fp16
-          const uint64_t bk = sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * ks, 16, 1024);
-          mma_ts(d1, tbase + C::T_W + 8 * ks, bk, id1, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_ss(dU, sdesc_sw128(sbase + C::S_W + 32 * ks, 16, 1024),
+                 sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * ks, 16, 1024), id1, ks > 0 ? 1u : 0u);
         mma_commit(bar(C::B_D1F + w));
+      };
+      int cnt = 0;
+      bool ok = w < ntiles && mbar_wait(bar(C::B_CVT + w), 0, abort_flag, err);
+      if (ok) {
+        tc_fence_after();
+        mma1(w);
+      }
+      for (int i = w; i < ntiles && ok; i += 2, ++cnt) {
+        const int s = i % C::NST;
+        if (i + 2 < ntiles) {
+          if (!mbar_wait(bar(C::B_UE + w), cnt & 1, abort_flag, err)) break;         // U^T of tile i read
+          if (!mbar_wait(bar(C::B_CVT + w), (cnt + 1) & 1, abort_flag, err)) break;  // tile i + 2 prepared
+          tc_fence_after();
+          mma1(i + 2);
+        }
         if (!mbar_wait(bar(C::B_PHI + w), cnt & 1, abort_flag, err)) break;
         tc_fence_after();
-        const uint32_t lbo = C::S_ONES - (C::S_V + s * C::TILE);  // V atom -> ones atom
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {  // MMA2: S_w += phi^T [V | 1]
-          const uint64_t bv = sdesc_sw128(sbase + C::S_V + s * C::TILE + 2048 * ks, lbo, 1024);
-          mma_ts(sw, d1 + 8 * ks, bv, idv, (cnt > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 8; ++ks) {  // MMA2: S_w += phi^T V, 16 tokens per step
+          const uint64_t bv = sdesc_sw128(sbase + C::S_V + s * C::TILE + 2048 * ks, 16, 1024);
+          mma_ts(dS, dP + 8 * ks, bv, idv, (cnt > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(bar(C::B_KVE + s));
         mma_commit(bar(C::B_SDONE + w));
@@ -563,14 +565,21 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       const int mine = (ntiles + 1 - w) / 2;
       if (mine > 0) mbar_wait(bar(C::B_SDONE + w), (mine - 1) & 1, abort_flag, err, 200000000ull);
     }
-  } else if (epi) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsHigh>();
     // ---------------- epilogue warpgroup ewg: tiles ewg, ewg + 2, ... ----------------
+    const int eq = warp & 3;
+    const int ewg = (warp - C::EPI0) >> 2;
+    const int frow = eq * 32 + lane;
+    const bool fvalid = frow < gw;
     // Each thread owns feature f0 + frow and reads each U^T value of its row once.  Its
     // stabiliser c is that feature's running max exponent over the tiles seen so far,
-    // raised (with an exact rescale of its S row) only when a tile exceeds it by more
-    // than 2^kTau, and never below floor = |w|^2 log2(e)/2 - 64: by completing the square
-    // no exponent of this feature exceeds |w|^2 log2(e)/2, so no phi exceeds 2^64 and the
-    // fp32 state cannot overflow for any |v| < 2^46 at any sequence length up to 2^17.
+    // raised (with an exact rescale of its S row and normaliser) only when a tile exceeds
+    // it by more than 2^kTau, and never below floor = |w|^2 log2(e)/2 - 64: by completing
+    // the square no exponent of this feature exceeds |w|^2 log2(e)/2, so no phi exceeds
+    // 2^64 and the fp32 state cannot overflow for any |v| < 2^46 at any sequence length up
+    // to 2^17.
     float floor_c;
     {
       float w2 = 0.f;
@@ -584,22 +593,20 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       }
       floor_c = w2 * static_cast<float>(kLog2e * 0.5) - 64.f;
     }
-    float c_run = floor_c, tmax = -INFINITY;
-    const uint32_t d1col = C::T_D1 + 128 * ewg;
-    const uint32_t scol = C::T_S + C::NS * ewg;
-    // Prepares tile i for its projection, one key row (token frow) per thread: stores -n(k) =
-    // -|k|^2 * nscale (-inf past the chunk end) and rewrites the bf16 row in place as fp16 times
-    // 2^-k, with one k per tile that puts the tile's largest |k| in [2^14, 2^15), so that the
-    // fp16 operand neither overflows nor loses the small values; returns 2^k.  The 16-byte
-    // chunks of a swizzled row are converted in place and summed in any order; thread frow starts
-    // at chunk frow % 8, so the eight threads of a shared-memory wavefront hit different banks.
-    int* red = reinterpret_cast<int*>(smem + C::S_RED) + 4 * ewg;
-    auto prepare_tile = [&](int i) -> float {
+    float c_run = floor_c, tmax = -INFINITY, zsum = 0.f;  // zsum: this feature's normaliser sum_t phi
+    const uint32_t cU = ewg * C::T_STRIDE + C::T_U, cP = ewg * C::T_STRIDE + C::T_P,
+                   cS = ewg * C::T_STRIDE + C::T_S;
+    // Prepares tile i for its projection, one key row (token frow) per thread: stores
+    // -n(k) = -|k|^2 nscale (-inf past the chunk end) and 2^s, and rewrites the bf16 row in
+    // place as fp16 times 2^-s, with s chosen from |k|^2 so that |k| 2^-s lies in [2^14, 2^15):
+    // no entry overflows fp16, and the largest keeps 11 bits.  The 16-byte chunks of a
+    // swizzled row are summed in any order; thread frow starts at chunk frow % 8, so the
+    // eight threads of a shared-memory wavefront hit different banks.
+    auto prepare_tile = [&](int i) {
       const int s = i % C::NST;
       mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err);
       uint4* row = reinterpret_cast<uint4*>(smem + C::S_K + s * C::TILE + frow * 128);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t emax = 0;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint4 v = row[c ^ (frow & 7)];
@@ -609,19 +616,18 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
           const float lo = __uint_as_float(wv[k] << 16), hi = __uint_as_float(wv[k] & 0xFFFF0000u);
           acc[k] = fmaf(lo, lo, acc[k]);
           acc[k] = fmaf(hi, hi, acc[k]);
-          emax = max(emax, max(wv[k] & 0x7F80u, (wv[k] >> 16) & 0x7F80u));
         }
       }
       const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-      nrm[s * 128 + frow] = (t_begin + 128 * i + frow < t_end) ? -sum * nscale : -INFINITY;
-      emax = __reduce_max_sync(0xffffffffu, emax);
-      if (lane == 0) red[eq] = static_cast<int>(emax >> 7);
-      named_bar_sync(1 + ewg, 128);
-      const int e = max(max(red[0], red[1]), max(red[2], red[3]));  // biased exponent of the tile max
-      const int k = min(100, max(-100, e - 141));                     // 2^(e-127) * 2^-k in [2^14, 2^15)
-      const float down = __int_as_float((127 - k) << 23);
+      // |k| < 2^((E+1)/2) <= 2^(floor(E/2)+1) for sum = |k|^2 in [2^E, 2^(E+1))
+      const int e2 = static_cast<int>((__float_as_uint(sum) >> 23) & 0xFF) - 127;
+      const int sh = min(100, max(-100, (e2 >> 1) + 1 - 15));
+      const bool inside = t_begin + 128 * i + frow < t_end;
+      nrm[s * 256 + frow] = inside ? -sum * nscale : -INFINITY;
+      nrm[s * 256 + 128 + frow] = __int_as_float((127 + sh) << 23);
+      const float down = __int_as_float((127 - sh) << 23);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {  // read again rather than hold 32 registers across the barrier
+      for (int c = 0; c < 8; ++c) {  // read again rather than hold 32 registers
         const uint4 v = row[c ^ (frow & 7)];
         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
         uint32_t o[4];
@@ -632,87 +638,97 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       }
       fence_proxy_async_smem();  // the converted row is read by the tensor cores
       named_bar_sync(1 + ewg, 128);
-      if (tid == C::EPI0 * 32 + 128 * ewg) mbar_arrive(bar(C::B_CVT + ewg));
-      return __int_as_float((127 + k) << 23);
+      if (eq == 0 && lane == 0) mbar_arrive(bar(C::B_CVT + ewg));
     };
     int cnt = 0;
-    float up_next = ewg < ntiles ? prepare_tile(ewg) : 1.f;
+    if (ewg < ntiles) prepare_tile(ewg);
     for (int i = ewg; i < ntiles; i += 2, ++cnt) {
-      const float up = up_next;
       const int s = i % C::NST;
       mbar_wait(bar(C::B_D1F + ewg), cnt & 1, abort_flag, err);
-      tc_fence_after();
-      // the previous tile raised the running max: rescale S now (its MMA2 has completed,
-      // since this tile's MMA1 was issued after it)
-      const bool need = tmax > c_run + kTau;
-      if (__any_sync(0xffffffffu, need)) scale_tmem_row(taddr(tbase, eq, scol), C::NS / 8, need ? ex2(c_run - tmax) : 1.f);
-      if (need) c_run = tmax;
-      const float cc_run = c_run;
-      const float4* nv = reinterpret_cast<const float4*>(nrm + s * 128);
-      uint32_t cur[32], nxt[32];
-      tmem_ld32(taddr(tbase, eq, d1col), cur);
+      // the projection of i + 2 is issued as soon as this tile's U^T has been read; preparing it
+      // only after U^T of i has arrived keeps each preparation one phase ahead of its consumer
+      if (i + 2 < ntiles) prepare_tile(i + 2);
+      // this tile's U^T row into registers (one read), then release it to the next projection
+      float ut[128];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(taddr(tbase, eq, cU + 32 * q4), *reinterpret_cast<uint32_t(*)[32]>(&ut[32 * q4]));
       tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_UE + ewg));
+      if (cnt >= 1) mbar_wait(bar(C::B_SDONE + ewg), (cnt - 1) & 1, abort_flag, err);  // phi buffer free, S final
+      tc_fence_after();
+      // the previous tile raised the running max: rescale S and the normaliser now
+      const bool need = tmax > c_run + kTau;
+      if (__any_sync(0xffffffffu, need)) scale_tmem_row(taddr(tbase, eq, cS), D / 8, need ? ex2(c_run - tmax) : 1.f);
+      if (need) {
+        zsum *= ex2(c_run - tmax);
+        c_run = tmax;
+      }
+      const float cc_run = c_run;
+      const float4* nv = reinterpret_cast<const float4*>(nrm + s * 256);
+      const float4* uv = reinterpret_cast<const float4*>(nrm + s * 256 + 128);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        if (q4 < 3) tmem_ld32(taddr(tbase, eq, d1col + 32 * (q4 + 1)), nxt);  // next chunk streams in meanwhile
         uint32_t wph[16];
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
           const float4 n4 = nv[8 * q4 + k4];
-          const float a0 = fmaf(__uint_as_float(cur[4 * k4 + 0]), up, n4.x);
-          const float a1 = fmaf(__uint_as_float(cur[4 * k4 + 1]), up, n4.y);
-          const float a2 = fmaf(__uint_as_float(cur[4 * k4 + 2]), up, n4.z);
-          const float a3 = fmaf(__uint_as_float(cur[4 * k4 + 3]), up, n4.w);
+          const float4 u4 = uv[8 * q4 + k4];
+          const float* r = &ut[32 * q4 + 4 * k4];
+          const float a0 = fmaf(r[0], u4.x, n4.x);
+          const float a1 = fmaf(r[1], u4.y, n4.y);
+          const float a2 = fmaf(r[2], u4.z, n4.z);
+          const float a3 = fmaf(r[3], u4.w, n4.w);
           tmax = max3(tmax, a0, a1);
           tmax = max3(tmax, a2, a3);
-          wph[2 * k4] = pack_bf16x2(ex2(a0 - cc_run), ex2(a1 - cc_run));
-          wph[2 * k4 + 1] = pack_bf16x2(ex2(a2 - cc_run), ex2(a3 - cc_run));
+          const float p0 = ex2(a0 - cc_run), p1 = ex2(a1 - cc_run), p2 = ex2(a2 - cc_run), p3 = ex2(a3 - cc_run);
+          zsum += (p0 + p1) + (p2 + p3);
+          wph[2 * k4] = pack_bf16x2(p0, p1);
+          wph[2 * k4 + 1] = pack_bf16x2(p2, p3);
         }
         if (!fvalid) {
 #pragma unroll
           for (int k = 0; k < 16; ++k) wph[k] = 0u;
         }
-        tmem_st16(taddr(tbase, eq, d1col + 16 * q4), wph);  // phi over columns already read
-        if (q4 < 3) {
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) cur[k] = nxt[k];
-        }
+        tmem_st16(taddr(tbase, eq, cP + 16 * q4), wph);  // phi, bf16 pairs
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_PHI + ewg));
-      if (i + 2 < ntiles) up_next = prepare_tile(i + 2);  // while this tile's MMA2 runs
     }
+    if (!fvalid) zsum = 0.f;
     // merge the two accumulators row by row and write this group's partial state
     cw[ewg * 128 + frow] = c_run;
+    cw[256 + ewg * 128 + frow] = zsum;
     named_bar_sync(3, 256);
+    const int n0 = (ntiles + 1) / 2, n1 = ntiles / 2;  // tiles of each warpgroup
     const float c0 = cw[frow], c1 = cw[128 + frow];
-    const bool has1 = cnt_of[1] > 0;
-    const float cmax = has1 ? fmaxf(c0, c1) : c0;
-    mbar_wait(bar(C::B_SDONE + 0), (cnt_of[0] - 1) & 1, abort_flag, err);
-    if (has1) mbar_wait(bar(C::B_SDONE + 1), (cnt_of[1] - 1) & 1, abort_flag, err);
+    const float cmax = n1 > 0 ? fmaxf(c0, c1) : c0;
+    if (n0 > 0) mbar_wait(bar(C::B_SDONE + 0), (n0 - 1) & 1, abort_flag, err);
+    if (n1 > 0) mbar_wait(bar(C::B_SDONE + 1), (n1 - 1) & 1, abort_flag, err);
     tc_fence_after();
-    const float s0 = ex2(c0 - cmax), s1 = has1 ? ex2(c1 - cmax) : 0.f;
+    const float s0 = n0 > 0 ? ex2(c0 - cmax) : 0.f, s1 = n1 > 0 ? ex2(c1 - cmax) : 0.f;
     float* outp = part_S + (static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * (D + 1);
 #pragma unroll
-    for (int cc = 0; cc < C::NS / 16; ++cc) {  // this warpgroup's half of the columns
-      const int col0 = ewg * (C::NS / 2) + 8 * cc;
+    for (int cc = 0; cc < D / 16; ++cc) {  // this warpgroup's half of the columns
+      const int col0 = ewg * (D / 2) + 8 * cc;
       uint32_t v0[8], v1[8];
       tmem_ld8(taddr(tbase, eq, C::T_S + col0), v0);
-      tmem_ld8(taddr(tbase, eq, C::T_S + C::NS + col0), v1);
+      tmem_ld8(taddr(tbase, eq, C::T_STRIDE + C::T_S + col0), v1);
       tmem_wait_ld();
       if (fvalid) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float v = __uint_as_float(v0[k]) * s0;
-          if (has1) v = fmaf(__uint_as_float(v1[k]), s1, v);
-          if (col0 + k <= D) outp[static_cast<size_t>(f0 + frow) * (D + 1) + col0 + k] = v;
-        }
+        for (int k = 0; k < 8; ++k)
+          outp[static_cast<size_t>(f0 + frow) * (D + 1) + col0 + k] =
+              fmaf(__uint_as_float(v1[k]), s1, __uint_as_float(v0[k]) * s0);
       }
     }
-    if (ewg == 0 && fvalid) part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + frow] = cmax;
+    if (ewg == 0 && fvalid) {
+      outp[static_cast<size_t>(f0 + frow) * (D + 1) + D] = fmaf(cw[384 + frow], s1, cw[256 + frow] * s0);
+      part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + frow] = cmax;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -729,16 +745,12 @@ struct QueryCfg {
   // warps 4-11 two epilogue warpgroups on alternate tiles
   static constexpr int THREADS = 384;
   static constexpr int EPI0 = 4;
-  // d = 64: the normaliser comes out of MMA2 as a ones column (N = d + 16); d = 128: two
-  // accumulators of d + 16 columns do not fit in tensor memory next to two U buffers, so
-  // MMA2 has N = d and the epilogue sums phi' s_f for the normaliser
-  static constexpr bool DEN_MMA = D == 64;
-  static constexpr int NO = DEN_MMA ? D + 16 : D;  // MMA2 N = rows of the state image
-  static constexpr int MMAX = D == 64 ? 512 : 256;  // features held in shared memory
+  static constexpr int FB = D == 64 ? 128 : 64;      // features per block (MMA1 N, MMA2 K)
+  static constexpr int MMAX = D == 64 ? 512 : 256;   // features held in shared memory
   static constexpr int QTILE = 128 * D * 2;
-  static constexpr int SP = NO * 128 * (MMAX / 64) + 8 * MMAX;  // fp16 image, exponents, fp32 normaliser column
-  // TMEM columns: warpgroup w owns U at w * TSTRIDE and O right after it
-  static constexpr int TSTRIDE = 128 + NO;
+  static constexpr int SP = D * 128 * (MMAX / 64) + 8 * MMAX;  // fp16 image, exponents, fp32 normaliser column
+  // TMEM columns: warpgroup w owns U at w * TSTRIDE, then phi' (FB / 2 columns of fp16 pairs), then O
+  static constexpr int TSTRIDE = FB + FB / 2 + D;
   static_assert(2 * TSTRIDE <= 512, "TMEM budget");
   // shared memory
   static constexpr int S_W = 0;                          // W' fp16, [D/64 regions][MMAX rows][128 B]
@@ -746,22 +758,24 @@ struct QueryCfg {
   static constexpr int S_Q = S_SP + SP;                  // Q stage w belongs to warpgroup w
   static constexpr int S_STG = S_Q + 2 * QTILE;          // output staging, one 64-column region, shared
   static constexpr int S_BAR = S_STG + 128 * 128;
-  static constexpr int B_QF = 0, B_QE = 2, B_CVT = 4, B_UF = 6, B_PHI = 8, B_M2 = 10, B_OF = 12, B_OE = 14,
-                       B_SF = 16, B_SE = 17, B_STG = 18, NBAR = 19;
+  static constexpr int B_QF = 0, B_QE = 2, B_CVT = 4, B_UF = 6, B_UE = 8, B_PHI = 10, B_M2 = 12, B_OF = 14,
+                       B_OE = 16, B_SF = 18, B_SE = 19, B_STG = 20, NBAR = 21;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int SMEM = S_ABORT + 16 + 1024;
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(S_SP % 1024 == 0 && S_Q % 1024 == 0 && S_STG % 1024 == 0 && (NO * 128) % 1024 == 0,
-                "128-byte swizzled operands start on 1024-byte boundaries");
+  static_assert(S_SP % 1024 == 0 && S_Q % 1024 == 0 && S_STG % 1024 == 0, "128-byte swizzled operands start on 1024-byte boundaries");
 };
 
 // Query pass.  The CTA's tiles go alternately to two epilogue warpgroups, each with its own
-// U buffer, O accumulator, Q stage and MMA-issuing thread, so one warpgroup's exponentials
-// overlap the other's tensor-memory reads, waits and output.  Per 128-feature block a
-// warpgroup reads U twice from tensor memory: once for the exact row max of 2^k U + e, once
-// to exponentiate; the row stabiliser is raised lazily across blocks with an exact rescale
-// of O.  The projection runs in fp16: each warpgroup rewrites its next Q tile in place as
+// U, phi' and O buffers in tensor memory, its own Q stage and its own MMA-issuing thread, so
+// one warpgroup's exponentials overlap the other's tensor-memory reads, waits and output.
+// Per block of FB features a warpgroup reads U twice: once for the exact row max of
+// 2^k U + e, once to exponentiate; as soon as the second read is done U is released, so the
+// next block's projection runs while this block's exponentials and contraction finish.  The
+// row stabiliser is raised lazily across blocks with an exact rescale of O and of the
+// normaliser, which the epilogue sums itself (phi' times the state's fp32 normaliser
+// column).  The projection runs in fp16: each warpgroup rewrites its next Q tile in place as
 // fp16 times 2^-k, one k per row that puts the row's largest |q| in [2^14, 2^15), and
 // multiplies that row's U by 2^k.
 template <int D>
@@ -771,6 +785,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     float wscale) {
   using C = QueryCfg<D>;
   constexpr int NT = C::THREADS;
+  constexpr int FB = C::FB;
   extern __shared__ unsigned char smem_raw[];
   // offset the __shared__ array itself (not via an integer cast), so that every pointer derived
   // from it stays a shared-memory pointer and compiles to shared loads and stores
@@ -779,7 +794,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ntq = (L + 127) / 128;
   const int G = H / Hkv;
-  const int nb = (m + 127) / 128;
+  const int nb = (m + FB - 1) / FB;
   const int per = ntiles_total / gridDim.x, extra = ntiles_total % gridDim.x;
   const int T0 = blockIdx.x * per + min(static_cast<int>(blockIdx.x), extra);
   const int n = per + (static_cast<int>(blockIdx.x) < extra ? 1 : 0);
@@ -802,6 +817,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       mbar_init(bar(C::B_QE + i), 1);
       mbar_init(bar(C::B_CVT + i), 1);
       mbar_init(bar(C::B_UF + i), 1);
+      mbar_init(bar(C::B_UE + i), 4);
       mbar_init(bar(C::B_PHI + i), 4);
       mbar_init(bar(C::B_M2 + i), 1);
       mbar_init(bar(C::B_OF + i), 1);
@@ -821,7 +837,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   }
   // W' in fp16 as the K-major, 128B-swizzled B operand of MMA1: row f, 16-byte chunk c at c ^ (f % 8)
   {
-    const int rows = nb * 128;
+    const int rows = nb * FB;
     constexpr int CPR = D / 8;  // 16-byte chunks per row
     for (int item = tid; item < rows * CPR; item += NT) {
       const int f = item / CPR, c = item % CPR;
@@ -847,7 +863,11 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   tc_fence_after();
   const uint32_t tbase = *tptr_slot;
   unsigned int* err = &g_sm100_error_word;
-
+  // registers: the producer / MMA warpgroup gives part of its share to the two epilogue
+  // warpgroups (128 x 96 + 256 x 200 = 63488 <= 384 x 168, the launch allocation; the host
+  // checks the compiled count before launching)
+  if (warp < C::EPI0) {
+  setmaxnreg_dec<kRegsLow>();
   if (warp == 0) {
     // ---------------- producer: Q tiles (stage = tile parity) and state images ----------------
     if (lane == 0) {
@@ -875,12 +895,17 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     }
   } else if (warp == 1 || warp == 2) {
     // ---------------- MMA issuer of warpgroup w = warp - 1: its tiles w, w + 2, ... ----------------
+    // Within a tile the next block's projection goes out as soon as the epilogue has read this
+    // block's U, ahead of this block's contraction; across tiles it waits for the next tile's
+    // Q, which the epilogue converts after handing over the tile's last block.
     if (lane == 0) {
       const int w = warp - 1;
-      const uint32_t id2 = idesc_f16(128, C::NO, false, false);
-      const uint32_t dU = tbase + w * C::TSTRIDE, dO = dU + 128;
+      const uint32_t id2 = idesc_f16(128, D, false, false);
+      const uint32_t dU = tbase + w * C::TSTRIDE, dP = dU + FB, dO = dP + FB / 2;
       const uint32_t qbase = sbase + C::S_Q + w * C::QTILE;
-      int cntb = 0, tc = 0, rel = 0;  // my blocks and tiles so far; images below rel released by me
+      const int ntw = (n - w + 1) / 2;  // my tiles
+      const int nblk = ntw * nb;        // my blocks
+      int rel = 0;                      // images below rel released by me
       bool ok = true;
       // releases image rel without having used it (after its predecessor's release completed,
       // so that the arrival counts towards the right phase)
@@ -890,63 +915,89 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         ++rel;
         return true;
       };
-      for (int t = w; t < n && ok; t += 2, ++tc) {
-        const int k = img(t);
-        while (rel < k && ok) ok = release_unused();
-        for (int j = 0; j < nb && ok; ++j, ++cntb) {
-          if (j == 0 && !mbar_wait(bar(C::B_CVT + w), tc & 1, abort_flag, err)) { ok = false; break; }
-          if (cntb >= 1 && !mbar_wait(bar(C::B_M2 + w), (cntb - 1) & 1, abort_flag, err)) { ok = false; break; }
-          tc_fence_after();
-          const int bw = min(128, m - 128 * j);
-          const uint32_t id1 = idesc_f16(128, bw, false, false);
+      auto mma1 = [&](int b) {  // U = (2^-k Q) W'^T in fp16 for my block b
+        const int j = b % nb, bw = min(FB, m - FB * j);
+        const uint32_t id1 = idesc_f16(128, bw, false, false);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {  // MMA1: U = (2^-k Q) W'^T in fp16
-            const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
-            const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (128 * j) * 128 + 32 * (ks & 3);
-            mma_ss(dU, sdesc_sw128(qbase + qo, 16, 1024), sdesc_sw128(sbase + C::S_W + wo, 16, 1024), id1,
-                   ks > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(C::B_UF + w));
-          if (j == nb - 1) mma_commit(bar(C::B_QE + w));  // the Q stage may take tile t + 2
-          if (!mbar_wait(bar(C::B_PHI + w), cntb & 1, abort_flag, err)) { ok = false; break; }
-          if (j == 0) {
-            if (tc >= 1 && !mbar_wait(bar(C::B_OE + w), (tc - 1) & 1, abort_flag, err)) { ok = false; break; }
-            if (!mbar_wait(bar(C::B_SF), k & 1, abort_flag, err)) { ok = false; break; }
-          }
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
+          const uint32_t wo = (ks >> 2) * (C::MMAX * 128) + (FB * j) * 128 + 32 * (ks & 3);
+          mma_ss(dU, sdesc_sw128(qbase + qo, 16, 1024), sdesc_sw128(sbase + C::S_W + wo, 16, 1024), id1,
+                 ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(C::B_UF + w));
+        if (j == nb - 1) mma_commit(bar(C::B_QE + w));  // the Q stage may take my next tile
+      };
+      // before the first projection of my tile tcn: release the images that precede its image
+      // and that I never used, then wait for its Q to be converted
+      auto enter_tile = [&](int tcn) {
+        const int kn = img(w + 2 * tcn);
+        while (rel < kn)
+          if (!release_unused()) return false;
+        return mbar_wait(bar(C::B_CVT + w), tcn & 1, abort_flag, err);
+      };
+      if (nblk > 0) {
+        ok = enter_tile(0);
+        if (ok) {
           tc_fence_after();
-          for (int ks = 0; ks < bw / 16; ++ks) {  // MMA2: O += phi' S', 16 features per step, two per TMEM column
-            const int fk = 128 * j + 16 * ks;
-            const uint64_t bd =
-                sdesc_sw128(sbase + C::S_SP + (fk >> 6) * (C::NO * 128) + 32 * ((fk & 63) >> 4), 16, 1024);
-            mma_ts(dO, dU + 8 * ks, bd, id2, (j > 0 || ks > 0) ? 1u : 0u);
+          mma1(0);
+        }
+      }
+      for (int b = 0; b < nblk && ok; ++b) {
+        const int tc = b / nb, j = b % nb, t = w + 2 * tc;
+        const int k = img(t);
+        const bool more = b + 1 < nblk, boundary = (j == nb - 1);
+        if (more && !boundary) {  // next block of the same tile
+          if (!mbar_wait(bar(C::B_UE + w), b & 1, abort_flag, err)) break;
+          tc_fence_after();
+          mma1(b + 1);
+        }
+        if (!mbar_wait(bar(C::B_PHI + w), b & 1, abort_flag, err)) break;
+        if (j == 0) {
+          if (tc >= 1 && !mbar_wait(bar(C::B_OE + w), (tc - 1) & 1, abort_flag, err)) break;
+          if (!mbar_wait(bar(C::B_SF), k & 1, abort_flag, err)) break;
+        }
+        tc_fence_after();
+        const int bw = min(FB, m - FB * j);
+        for (int ks = 0; ks < bw / 16; ++ks) {  // MMA2: O += phi' S', 16 features per step, two per TMEM column
+          const int fk = FB * j + 16 * ks;
+          const uint64_t bd = sdesc_sw128(sbase + C::S_SP + (fk >> 6) * (D * 128) + 32 * ((fk & 63) >> 4), 16, 1024);
+          mma_ts(dO, dP + 8 * ks, bd, id2, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(C::B_M2 + w));
+        if (boundary) {
+          mma_commit(bar(C::B_OF + w));
+          const int knext = t + 2 < n ? img(t + 2) : nimg;
+          if (knext > k && k < nimg - 1) {  // done with image k: released when these MMAs complete
+            mma_commit(bar(C::B_SE));
+            rel = k + 1;
           }
-          mma_commit(bar(C::B_M2 + w));
-          if (j == nb - 1) {
-            mma_commit(bar(C::B_OF + w));
-            const int knext = t + 2 < n ? img(t + 2) : nimg;
-            if (knext > k && k < nimg - 1) {  // done with image k: released when these MMAs complete
-              mma_commit(bar(C::B_SE));
-              rel = k + 1;
-            }
+          if (more) {  // first block of my next tile: U read and that tile's Q converted
+            if (!mbar_wait(bar(C::B_UE + w), b & 1, abort_flag, err)) break;
+            if (!enter_tile(tc + 1)) break;
+            tc_fence_after();
+            mma1(b + 1);
           }
         }
       }
       while (ok && rel < nimg - 1) ok = release_unused();
-      if (cntb >= 1) mbar_wait(bar(C::B_M2 + w), (cntb - 1) & 1, abort_flag, err, 200000000ull);
+      if (nblk >= 1) mbar_wait(bar(C::B_M2 + w), (nblk - 1) & 1, abort_flag, err, 200000000ull);
     }
-  } else if (warp >= C::EPI0) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsHigh>();
     // ---------------- epilogue warpgroup ewg: tiles ewg, ewg + 2, ... ----------------
     const int eq = warp & 3;
     const int ewg = (warp - C::EPI0) >> 2;
     const int r = eq * 32 + lane;  // query row within the tile (TMEM lane)
     const bool issuer = (eq == 0 && lane == 0);
-    const uint32_t cU = ewg * C::TSTRIDE, cO = cU + 128;  // TMEM columns
-    const int atoms = (m + 63) / 64;  // the image holds [atoms][NO rows][64 features] fp16, then its tail
-    const float* ev = reinterpret_cast<const float*>(smem + C::S_SP + C::NO * 128 * atoms);
+    const uint32_t cU = ewg * C::TSTRIDE, cP = cU + FB, cO = cP + FB / 2;  // TMEM columns
+    const int atoms = (m + 63) / 64;  // the image holds [atoms][D rows][64 features] fp16, then its tail
+    const float* ev = reinterpret_cast<const float*>(smem + C::S_SP + D * 128 * atoms);
     const float* sd = ev + 64 * atoms;  // fp32 normaliser column of the state, same scaling as the image
     // rewrites row r of Q tile t (Q stage ewg) as fp16 x 2^-k; returns 2^k.  Thread r starts at
     // chunk r % 8 so that the eight threads of a shared-memory wavefront hit different banks.
-    auto prepare = [&](int t, int tcount) -> float {
+    auto prepare = [&](int tcount) -> float {
       mbar_wait(bar(C::B_QF + ewg), tcount & 1, abort_flag, err);
       unsigned char* qrow = smem + C::S_Q + ewg * C::QTILE + r * 128;
       uint32_t emax = 0;
@@ -979,7 +1030,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       if (issuer) mbar_arrive(bar(C::B_CVT + ewg));
       return __int_as_float((127 + k) << 23);
     };
-    float up_next = ewg < n ? prepare(ewg, 0) : 1.f;
+    float up_next = ewg < n ? prepare(0) : 1.f;
     int cntb = 0, tc = 0;
     for (int t = ewg; t < n; t += 2, ++tc) {
       const float up = up_next;
@@ -988,87 +1039,58 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       for (int j = 0; j < nb; ++j, ++cntb) {
         mbar_wait(bar(C::B_UF + ewg), cntb & 1, abort_flag, err);
         tc_fence_after();
-        const float4* e4p = reinterpret_cast<const float4*>(ev + 128 * j);
-        const bool ragged = 128 * j + 128 > m;  // features past m in this block (warp-uniform)
-        // pass 1: row max of 2^k U + e over the block
-        float mx;
-        {
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          uint32_t cur[32], nxt[32];
-          tmem_ld32(taddr(tbase, eq, cU), cur);
-          tmem_wait_ld();
+        // the whole block of this row into registers: one read of U, which is then released
+        float v[FB];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            if (q4 < 3) tmem_ld32(taddr(tbase, eq, cU + 32 * (q4 + 1)), nxt);
+        for (int q4 = 0; q4 < FB / 32; ++q4) tmem_ld32(taddr(tbase, eq, cU + 32 * q4), *reinterpret_cast<uint32_t(*)[32]>(&v[32 * q4]));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_UE + ewg));  // the next projection may overwrite U
+        const float4* e4p = reinterpret_cast<const float4*>(ev + FB * j);
+        const float4* s4p = reinterpret_cast<const float4*>(sd + FB * j);
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-              const float4 e4 = e4p[8 * q4 + k4];
-              float a[4] = {fmaf(__uint_as_float(cur[4 * k4 + 0]), up, e4.x),
-                            fmaf(__uint_as_float(cur[4 * k4 + 1]), up, e4.y),
-                            fmaf(__uint_as_float(cur[4 * k4 + 2]), up, e4.z),
-                            fmaf(__uint_as_float(cur[4 * k4 + 3]), up, e4.w)};
-              if (ragged) {
+        for (int k4 = 0; k4 < FB / 4; ++k4) {  // 2^k U + e and its row max
+          const float4 e4 = e4p[k4];
+          v[4 * k4 + 0] = fmaf(v[4 * k4 + 0], up, e4.x);
+          v[4 * k4 + 1] = fmaf(v[4 * k4 + 1], up, e4.y);
+          v[4 * k4 + 2] = fmaf(v[4 * k4 + 2], up, e4.z);
+          v[4 * k4 + 3] = fmaf(v[4 * k4 + 3], up, e4.w);
+          if (FB * j + FB > m) {  // features past m (a warp-uniform condition)
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  if (128 * j + 32 * q4 + 4 * k4 + e >= m) a[e] = -INFINITY;
-              }
-              m4[k4 & 3] = max3(m4[k4 & 3], a[0], a[1]);
-              m4[k4 & 3] = max3(m4[k4 & 3], a[2], a[3]);
-            }
-            if (q4 < 3) {
-              tmem_wait_ld();
-#pragma unroll
-              for (int k = 0; k < 32; ++k) cur[k] = nxt[k];
-            }
+            for (int e = 0; e < 4; ++e)
+              if (FB * j + 4 * k4 + e >= m) v[4 * k4 + e] = -INFINITY;
           }
-          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          m4[k4 & 3] = max3(m4[k4 & 3], v[4 * k4 + 0], v[4 * k4 + 1]);
+          m4[k4 & 3] = max3(m4[k4 & 3], v[4 * k4 + 2], v[4 * k4 + 3]);
         }
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        // the previous block's contraction must be complete before phi' is overwritten or O rescaled
+        if (cntb >= 1) mbar_wait(bar(C::B_M2 + ewg), (cntb - 1) & 1, abort_flag, err);
+        tc_fence_after();
         const bool need = (j > 0) && (mx > c + kTau);
         if (j == 0) c = mx;
         if (__any_sync(0xffffffffu, need)) {  // raise the stabiliser of the rows that need it
-          mbar_wait(bar(C::B_M2 + ewg), (cntb - 1) & 1, abort_flag, err);  // O holds the previous blocks
-          tc_fence_after();
           const float f = need ? ex2(c - mx) : 1.f;
-          scale_tmem_row(taddr(tbase, eq, cO), C::NO / 8, f);
+          scale_tmem_row(taddr(tbase, eq, cO), D / 8, f);
           den *= f;
         }
         if (need) c = mx;
-        // pass 2: phi' = 2^(2^k U + e - c) as fp16 over the first 64 columns of U
-        {
-          uint32_t cur[32], nxt[32];
-          tmem_ld32(taddr(tbase, eq, cU), cur);
-          tmem_wait_ld();
+        // phi' = 2^(2^k U + e - c) as fp16 pairs into the phi' buffer; normaliser in fp32
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            if (q4 < 3) tmem_ld32(taddr(tbase, eq, cU + 32 * (q4 + 1)), nxt);
-            uint32_t ph[16];
+        for (int q4 = 0; q4 < FB / 32; ++q4) {
+          uint32_t ph[16];
 #pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-              const float4 e4 = e4p[8 * q4 + k4];
-              float a[4] = {fmaf(__uint_as_float(cur[4 * k4 + 0]), up, e4.x),
-                            fmaf(__uint_as_float(cur[4 * k4 + 1]), up, e4.y),
-                            fmaf(__uint_as_float(cur[4 * k4 + 2]), up, e4.z),
-                            fmaf(__uint_as_float(cur[4 * k4 + 3]), up, e4.w)};
-              if (ragged) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  if (128 * j + 32 * q4 + 4 * k4 + e >= m) a[e] = -INFINITY;
-              }
-              const float p0 = ex2(a[0] - c), p1 = ex2(a[1] - c), p2 = ex2(a[2] - c), p3 = ex2(a[3] - c);
-              if constexpr (!C::DEN_MMA) {
-                const float4 s4 = reinterpret_cast<const float4*>(sd + 128 * j)[8 * q4 + k4];
-                den = fmaf(p0, s4.x, fmaf(p1, s4.y, fmaf(p2, s4.z, fmaf(p3, s4.w, den))));
-              }
-              ph[2 * k4] = pack_f16x2(p0, p1);
-              ph[2 * k4 + 1] = pack_f16x2(p2, p3);
-            }
-            tmem_st16(taddr(tbase, eq, cU + 16 * q4), ph);  // phi' over columns already read
-            if (q4 < 3) {
-              tmem_wait_ld();
-#pragma unroll
-              for (int k = 0; k < 32; ++k) cur[k] = nxt[k];
-            }
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 s4 = s4p[8 * q4 + k4];
+            const float* a = &v[32 * q4 + 4 * k4];
+            const float p0 = ex2(a[0] - c), p1 = ex2(a[1] - c), p2 = ex2(a[2] - c), p3 = ex2(a[3] - c);
+            den = fmaf(p0, s4.x, fmaf(p1, s4.y, fmaf(p2, s4.z, fmaf(p3, s4.w, den))));
+            ph[2 * k4] = pack_f16x2(p0, p1);
+            ph[2 * k4 + 1] = pack_f16x2(p2, p3);
           }
+          tmem_st16(taddr(tbase, eq, cP + 16 * q4), ph);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -1076,16 +1098,10 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         if (lane == 0) mbar_arrive(bar(C::B_PHI + ewg));
       }
       // the tile's blocks are handed over: convert the next tile's Q while the last MMA2 runs
-      if (t + 2 < n) up_next = prepare(t + 2, tc + 1);
-      // out = O[:, :d] / den -> bf16 -> shared staging (taken in tile order) -> TMA store
+      if (t + 2 < n) up_next = prepare(tc + 1);
+      // out = O / den -> bf16 -> shared staging (taken in tile order) -> TMA store
       mbar_wait(bar(C::B_OF + ewg), tc & 1, abort_flag, err);
       tc_fence_after();
-      if constexpr (C::DEN_MMA) {
-        uint32_t dv;
-        tmem_ld1(taddr(tbase, eq, cO + D), dv);
-        tmem_wait_ld();
-        den = __uint_as_float(dv);
-      }
       const float inv = 1.f / den;
       if (t >= 1) mbar_wait(bar(C::B_STG), (t - 1) & 1, abort_flag, err);  // tile t - 1 released the staging tile
       const int T = T0 + t, bh = T / ntq, qt = T % ntq;
@@ -1180,6 +1196,21 @@ int num_sms() {
   return sms > 0 ? sms : 1;
 }
 
+// The kernels that rebalance registers between warpgroups (setmaxnreg) need the launch to
+// hold at least what the rebalanced warpgroups ask for, or the increase would never be
+// granted: check the compiled register count once per kernel before the first launch.
+int check_register_split(const void* kern, int threads) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 kernel attributes: %s", cudaGetErrorString(e));
+  const long have = static_cast<long>(fa.numRegs) * threads;
+  const long need = 128L * kRegsLow + static_cast<long>(threads - 128) * kRegsHigh;
+  if (have < need)
+    return set_errorf(FAVOR_ERR_UNSUPPORTED, "sm100 kernel compiled with %d registers per thread: %ld < %ld needed",
+                      fa.numRegs, have, need);
+  return FAVOR_OK;
+}
+
 template <int D>
 int launch_key(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st) {
   CUtensorMap mk, mv;
@@ -1190,6 +1221,10 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   auto kern = (D == 64) ? key_pass_pp_sm100 : key_pass_sm100<D>;
   const int smem_bytes = (D == 64) ? KeyPP::SMEM : KeyCfg<D>::SMEM;
   const int threads = (D == 64) ? KeyPP::THREADS : kThreads;
+  if (D == 64) {
+    static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), threads);
+    if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), threads);
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass attribute: %s", cudaGetErrorString(e));
   char* base = static_cast<char*>(partials);
@@ -1211,6 +1246,8 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   if (rc == FAVOR_OK) rc = make_map(&mo, out, D, p.L, bh);
   if (rc != FAVOR_OK) return rc;
   auto kern = query_pass_sm100<D>;
+  static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), C::THREADS);
+  if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), C::THREADS);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass attribute: %s", cudaGetErrorString(e));
   const int ntiles = bh * ((p.L + 127) / 128);
