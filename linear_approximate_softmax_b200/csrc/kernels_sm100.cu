@@ -56,7 +56,7 @@ constexpr int kEpiThreads = 256;
 constexpr uint32_t kBarEpi = 1;    // named barrier: epilogue max exchange (lock-step key pass)
 constexpr float kTau = 8.f;        // lazy stabiliser threshold (log2 units)
 // registers per thread after setmaxnreg: producer / MMA warpgroup, epilogue warpgroups
-constexpr int kRegsLow = 96, kRegsHigh = 200;
+constexpr int kRegsLow = 88, kRegsHigh = 200;
 
 __device__ __forceinline__ uint32_t taddr(uint32_t base, int lane_quarter, int col) {
   return base + (static_cast<uint32_t>(lane_quarter * 32) << 16) + static_cast<uint32_t>(col);
@@ -461,7 +461,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       mbar_init(bar(C::B_KVE + s), 1);
     }
     for (int w = 0; w < 2; ++w) {
-      mbar_init(bar(C::B_CVT + w), 1);
+      mbar_init(bar(C::B_CVT + w), 4);  // one arrival per epilogue warp
       mbar_init(bar(C::B_D1F + w), 1);
       mbar_init(bar(C::B_UE + w), 4);
       mbar_init(bar(C::B_PHI + w), 4);
@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
   unsigned int* err = &g_sm100_error_word;
 
   // registers: the producer / MMA warpgroup gives part of its share to the two epilogue
-  // warpgroups (128 x 96 + 256 x 200 = 63488 <= 384 x 168, the launch allocation; the host
+  // warpgroups (128 x 88 + 256 x 200 = 62464 <= 384 x 168, the launch allocation; the host
   // checks the compiled count before launching)
   if (warp < C::EPI0) {
   setmaxnreg_dec<kRegsLow>();
@@ -637,14 +637,17 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
         row[c ^ (frow & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
       }
       fence_proxy_async_smem();  // the converted row is read by the tensor cores
-      named_bar_sync(1 + ewg, 128);
-      if (eq == 0 && lane == 0) mbar_arrive(bar(C::B_CVT + ewg));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_CVT + ewg));  // this warp's 32 rows are ready
     };
     int cnt = 0;
     if (ewg < ntiles) prepare_tile(ewg);
     for (int i = ewg; i < ntiles; i += 2, ++cnt) {
       const int s = i % C::NST;
       mbar_wait(bar(C::B_D1F + ewg), cnt & 1, abort_flag, err);
+      // every warp's norms of tile i are visible once all four have arrived for it (this
+      // warp waits before arriving for tile i + 2, so the phase cannot have moved on)
+      mbar_wait(bar(C::B_CVT + ewg), cnt & 1, abort_flag, err);
       // the projection of i + 2 is issued as soon as this tile's U^T has been read; preparing it
       // only after U^T of i has arrived keeps each preparation one phase ahead of its consumer
       if (i + 2 < ntiles) prepare_tile(i + 2);
@@ -665,27 +668,27 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
         zsum *= ex2(c_run - tmax);
         c_run = tmax;
       }
-      const float cc_run = c_run;
+      const float2 ncc = make_float2(-c_run, -c_run);
+      float2 zs2 = make_float2(0.f, 0.f);
       const float4* nv = reinterpret_cast<const float4*>(nrm + s * 256);
       const float4* uv = reinterpret_cast<const float4*>(nrm + s * 256 + 128);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t wph[16];
 #pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
+        for (int k4 = 0; k4 < 8; ++k4) {  // two tokens per packed fp32x2 operation
           const float4 n4 = nv[8 * q4 + k4];
           const float4 u4 = uv[8 * q4 + k4];
           const float* r = &ut[32 * q4 + 4 * k4];
-          const float a0 = fmaf(r[0], u4.x, n4.x);
-          const float a1 = fmaf(r[1], u4.y, n4.y);
-          const float a2 = fmaf(r[2], u4.z, n4.z);
-          const float a3 = fmaf(r[3], u4.w, n4.w);
-          tmax = max3(tmax, a0, a1);
-          tmax = max3(tmax, a2, a3);
-          const float p0 = ex2(a0 - cc_run), p1 = ex2(a1 - cc_run), p2 = ex2(a2 - cc_run), p3 = ex2(a3 - cc_run);
-          zsum += (p0 + p1) + (p2 + p3);
-          wph[2 * k4] = pack_bf16x2(p0, p1);
-          wph[2 * k4 + 1] = pack_bf16x2(p2, p3);
+          const float2 a01 = __ffma2_rn(make_float2(r[0], r[1]), make_float2(u4.x, u4.y), make_float2(n4.x, n4.y));
+          const float2 a23 = __ffma2_rn(make_float2(r[2], r[3]), make_float2(u4.z, u4.w), make_float2(n4.z, n4.w));
+          tmax = max3(tmax, a01.x, a01.y);
+          tmax = max3(tmax, a23.x, a23.y);
+          const float2 b01 = __fadd2_rn(a01, ncc), b23 = __fadd2_rn(a23, ncc);
+          const float2 p01 = make_float2(ex2(b01.x), ex2(b01.y)), p23 = make_float2(ex2(b23.x), ex2(b23.y));
+          zs2 = __fadd2_rn(zs2, __fadd2_rn(p01, p23));
+          wph[2 * k4] = pack_bf16x2(p01.x, p01.y);
+          wph[2 * k4 + 1] = pack_bf16x2(p23.x, p23.y);
         }
         if (!fvalid) {
 #pragma unroll
@@ -693,6 +696,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
         }
         tmem_st16(taddr(tbase, eq, cP + 16 * q4), wph);  // phi, bf16 pairs
       }
+      zsum += zs2.x + zs2.y;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -815,7 +819,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(C::B_QF + i), 1);
       mbar_init(bar(C::B_QE + i), 1);
-      mbar_init(bar(C::B_CVT + i), 1);
+      mbar_init(bar(C::B_CVT + i), 4);  // one arrival per epilogue warp
       mbar_init(bar(C::B_UF + i), 1);
       mbar_init(bar(C::B_UE + i), 4);
       mbar_init(bar(C::B_PHI + i), 4);
@@ -864,7 +868,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   const uint32_t tbase = *tptr_slot;
   unsigned int* err = &g_sm100_error_word;
   // registers: the producer / MMA warpgroup gives part of its share to the two epilogue
-  // warpgroups (128 x 96 + 256 x 200 = 63488 <= 384 x 168, the launch allocation; the host
+  // warpgroups (128 x 88 + 256 x 200 = 62464 <= 384 x 168, the launch allocation; the host
   // checks the compiled count before launching)
   if (warp < C::EPI0) {
   setmaxnreg_dec<kRegsLow>();
@@ -1026,8 +1030,8 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
           *p = make_uint4(o[0], o[1], o[2], o[3]);
         }
       fence_proxy_async_smem();  // the converted tile is read by the tensor cores
-      named_bar_sync(1 + ewg, 128);
-      if (issuer) mbar_arrive(bar(C::B_CVT + ewg));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_CVT + ewg));  // this warp's 32 rows are ready
       return __int_as_float((127 + k) << 23);
     };
     float up_next = ewg < n ? prepare(0) : 1.f;
@@ -1050,13 +1054,16 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         const float4* e4p = reinterpret_cast<const float4*>(ev + FB * j);
         const float4* s4p = reinterpret_cast<const float4*>(sd + FB * j);
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const float2 up2 = make_float2(up, up);
 #pragma unroll
-        for (int k4 = 0; k4 < FB / 4; ++k4) {  // 2^k U + e and its row max
+        for (int k4 = 0; k4 < FB / 4; ++k4) {  // 2^k U + e and its row max, two features per fp32x2 operation
           const float4 e4 = e4p[k4];
-          v[4 * k4 + 0] = fmaf(v[4 * k4 + 0], up, e4.x);
-          v[4 * k4 + 1] = fmaf(v[4 * k4 + 1], up, e4.y);
-          v[4 * k4 + 2] = fmaf(v[4 * k4 + 2], up, e4.z);
-          v[4 * k4 + 3] = fmaf(v[4 * k4 + 3], up, e4.w);
+          const float2 v01 = __ffma2_rn(make_float2(v[4 * k4 + 0], v[4 * k4 + 1]), up2, make_float2(e4.x, e4.y));
+          const float2 v23 = __ffma2_rn(make_float2(v[4 * k4 + 2], v[4 * k4 + 3]), up2, make_float2(e4.z, e4.w));
+          v[4 * k4 + 0] = v01.x;
+          v[4 * k4 + 1] = v01.y;
+          v[4 * k4 + 2] = v23.x;
+          v[4 * k4 + 3] = v23.y;
           if (FB * j + FB > m) {  // features past m (a warp-uniform condition)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -1078,6 +1085,8 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         }
         if (need) c = mx;
         // phi' = 2^(2^k U + e - c) as fp16 pairs into the phi' buffer; normaliser in fp32
+        const float2 nc2 = make_float2(-c, -c);
+        float2 den2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int q4 = 0; q4 < FB / 32; ++q4) {
           uint32_t ph[16];
@@ -1085,13 +1094,16 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
           for (int k4 = 0; k4 < 8; ++k4) {
             const float4 s4 = s4p[8 * q4 + k4];
             const float* a = &v[32 * q4 + 4 * k4];
-            const float p0 = ex2(a[0] - c), p1 = ex2(a[1] - c), p2 = ex2(a[2] - c), p3 = ex2(a[3] - c);
-            den = fmaf(p0, s4.x, fmaf(p1, s4.y, fmaf(p2, s4.z, fmaf(p3, s4.w, den))));
-            ph[2 * k4] = pack_f16x2(p0, p1);
-            ph[2 * k4 + 1] = pack_f16x2(p2, p3);
+            const float2 b01 = __fadd2_rn(make_float2(a[0], a[1]), nc2), b23 = __fadd2_rn(make_float2(a[2], a[3]), nc2);
+            const float2 p01 = make_float2(ex2(b01.x), ex2(b01.y)), p23 = make_float2(ex2(b23.x), ex2(b23.y));
+            den2 = __ffma2_rn(p01, make_float2(s4.x, s4.y), den2);
+            den2 = __ffma2_rn(p23, make_float2(s4.z, s4.w), den2);
+            ph[2 * k4] = pack_f16x2(p01.x, p01.y);
+            ph[2 * k4 + 1] = pack_f16x2(p23.x, p23.y);
           }
           tmem_st16(taddr(tbase, eq, cP + 16 * q4), ph);
         }
+        den += den2.x + den2.y;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
