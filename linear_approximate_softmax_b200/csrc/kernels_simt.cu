@@ -153,10 +153,13 @@ __global__ void __launch_bounds__(kThreads) key_pass_kernel(
 
 // grid (op_atoms * 64 / 32, B*Hkv), 256 threads: 32 feature rows per CTA, 8 threads
 // per row.  Each row is the sum of the chunk partials in the fixed order p = 0..P-1,
-// each rescaled from its own stabiliser to the head's largest one (bitwise
-// deterministic).  Writes S[f][n] (fp32), and the fp16 operand image of the query
-// pass: the row scaled by 2^-e[f] so that its largest entry lies in [2^14, 2^15)
-// (exact power-of-two scaling), zeros in the padding, and e[f].
+// each rescaled from its own stabiliser to the row's largest one c_f (bitwise
+// deterministic).  Writes S[f][n] = 2^(c_f - c*) x that sum (fp32, relative to the head's
+// largest stabiliser c*), c*, and the fp16 operand image of the query pass: the row
+// relative to c_f scaled by 2^-x_f so that its largest entry lies in [2^14, 2^15), then
+// e_f = x_f + (c_f - c*) and the normaliser entry with the same scaling.  Because the
+// image carries c_f - c* in e_f rather than in its fp16 values, a feature whose keys sit
+// far below the head's largest exponent keeps its precision on the query side.
 __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
     const float* __restrict__ part_S, const float* __restrict__ part_c, float* __restrict__ S,
     float* __restrict__ Sc, unsigned char* __restrict__ op, int P, int m, int D1, int nsb, int op_rows,
@@ -176,25 +179,35 @@ __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
 
   const int f = blockIdx.x * 32 + (threadIdx.x >> 3);  // feature row (< op_atoms * 64)
   const int g = threadIdx.x & 7;                       // this thread's columns: g, g + 8, ...
+  const bool live = f < m;
   constexpr int kMaxCols = (128 + 16) / 8;             // max(op_rows, D1) <= 144
   float val[kMaxCols];
+#pragma unroll
+  for (int k = 0; k < kMaxCols; ++k) val[k] = 0.f;
+  float cf = -INFINITY;  // this feature's largest chunk stabiliser
+  if (live)
+    for (int p = 0; p < P; ++p) cf = fmaxf(cf, pc[p * nsb + f / kStabBlock]);
+  if (cf > -INFINITY) {
+    for (int p = 0; p < P; ++p) {
+      const float c = pc[p * nsb + f / kStabBlock];
+      if (c == -INFINITY) continue;
+      const float wp = exp2f(c - cf);
+      const float* src = part_S + ((static_cast<size_t>(head) * P + p) * m + f) * D1;
+#pragma unroll
+      for (int k = 0; k < kMaxCols; ++k) {
+        const int n = g + 8 * k;
+        if (n < D1) val[k] = fmaf(wp, src[n], val[k]);
+      }
+    }
+  }
+  const float rel = cf > -INFINITY ? exp2f(cf - cs) : 0.f;  // the row relative to c*
   float amax = 0.f, den = 0.f;
 #pragma unroll
   for (int k = 0; k < kMaxCols; ++k) {
     const int n = g + 8 * k;
-    float acc = 0.f;
-    if (f < m && n < D1) {
-      const size_t idx = static_cast<size_t>(f) * D1 + n;
-      for (int p = 0; p < P; ++p) {
-        const float c = pc[p * nsb + f / kStabBlock];
-        const float wp = (c == -INFINITY) ? 0.f : exp2f(c - cs);
-        acc = fmaf(wp, part_S[(static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * D1 + idx], acc);
-      }
-      S[static_cast<size_t>(head) * m * D1 + idx] = acc;
-    }
-    val[k] = acc;
-    if (n < op_rows) amax = fmaxf(amax, fabsf(acc));
-    if (n == D1 - 1) den = acc;
+    if (live && n < D1) S[(static_cast<size_t>(head) * m + f) * D1 + n] = val[k] * rel;
+    if (n < op_rows) amax = fmaxf(amax, fabsf(val[k]));
+    if (n == D1 - 1) den = val[k];
   }
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
@@ -217,7 +230,7 @@ __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
   }
   // tail: the exponent of each feature, then its normaliser entry with the same scaling
   float* tail = reinterpret_cast<float*>(img + static_cast<size_t>(op_rows) * 128 * op_atoms);
-  if (g == 0) tail[f] = static_cast<float>(ex);
+  if (g == 0) tail[f] = live && cf > -INFINITY ? static_cast<float>(ex) + (cf - cs) : 0.f;
   if (((D1 - 1) & 7) == g) tail[64 * op_atoms + f] = ldexpf(den, -ex);
 }
 

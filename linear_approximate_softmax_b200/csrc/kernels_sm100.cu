@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % C::NST;
-        if (i >= C::NST && !mbar_wait(bar(C::B_KVE + s), ((i / C::NST) - 1) & 1, abort_flag, err)) break;
+        if (i >= C::NST && !mbar_wait<true>(bar(C::B_KVE + s), ((i / C::NST) - 1) & 1, abort_flag, err)) break;
         mbar_arrive_expect_tx(bar(C::B_KVF + s), 2 * C::TILE);
         const int t0 = t_begin + 128 * i;
         tma_load_3d(sbase + C::S_K + s * C::TILE, &tmK, bar(C::B_KVF + s), 0, t0, head);
@@ -598,43 +598,54 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
                    cS = ewg * C::T_STRIDE + C::T_S;
     // Prepares tile i for its projection, one key row (token frow) per thread: stores
     // -n(k) = -|k|^2 nscale (-inf past the chunk end) and 2^s, and rewrites the bf16 row in
-    // place as fp16 times 2^-s, with s chosen from |k|^2 so that |k| 2^-s lies in [2^14, 2^15):
-    // no entry overflows fp16, and the largest keeps 11 bits.  The 16-byte chunks of a
-    // swizzled row are summed in any order; thread frow starts at chunk frow % 8, so the
-    // eight threads of a shared-memory wavefront hit different banks.
+    // place as fp16 times 2^-s.  s = 0 unless |k| >= 2^15, when it brings |k| 2^-s into
+    // [2^14, 2^15) so that no entry overflows fp16; an entry below fp16's normal range keeps an
+    // absolute error under 2^-25, which moves an exponent by less than |w'|_1 2^-25.  The
+    // 16-byte chunks of a swizzled row are summed in any order; thread frow starts at chunk
+    // frow % 8, so the eight threads of a shared-memory wavefront hit different banks.
     auto prepare_tile = [&](int i) {
       const int s = i % C::NST;
       mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err);
       uint4* row = reinterpret_cast<uint4*>(smem + C::S_K + s * C::TILE + frow * 128);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      uint4 v[8];
+      float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const uint4 v = row[c ^ (frow & 7)];
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        v[c] = row[c ^ (frow & 7)];
+        const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float lo = __uint_as_float(wv[k] << 16), hi = __uint_as_float(wv[k] & 0xFFFF0000u);
-          acc[k] = fmaf(lo, lo, acc[k]);
-          acc[k] = fmaf(hi, hi, acc[k]);
+          const float2 x = make_float2(__uint_as_float(wv[k] << 16), __uint_as_float(wv[k] & 0xFFFF0000u));
+          acc[k & 1] = __ffma2_rn(x, x, acc[k & 1]);
         }
       }
-      const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      const float sum = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
       // |k| < 2^((E+1)/2) <= 2^(floor(E/2)+1) for sum = |k|^2 in [2^E, 2^(E+1))
       const int e2 = static_cast<int>((__float_as_uint(sum) >> 23) & 0xFF) - 127;
-      const int sh = min(100, max(-100, (e2 >> 1) + 1 - 15));
+      const int sh = min(100, max(0, (e2 >> 1) + 1 - 15));
       const bool inside = t_begin + 128 * i + frow < t_end;
       nrm[s * 256 + frow] = inside ? -sum * nscale : -INFINITY;
       nrm[s * 256 + 128 + frow] = __int_as_float((127 + sh) << 23);
-      const float down = __int_as_float((127 - sh) << 23);
+      if (__all_sync(0xffffffffu, sh == 0)) {  // the usual case: a plain conversion
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {  // read again rather than hold 32 registers
-        const uint4 v = row[c ^ (frow & 7)];
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-        uint32_t o[4];
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+          uint32_t o[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          o[q] = pack_f16x2(__uint_as_float(wv[q] << 16) * down, __uint_as_float(wv[q] & 0xFFFF0000u) * down);
-        row[c ^ (frow & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
+          for (int q = 0; q < 4; ++q) o[q] = pack_f16x2(__uint_as_float(wv[q] << 16), __uint_as_float(wv[q] & 0xFFFF0000u));
+          row[c ^ (frow & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      } else {
+        const float down = __int_as_float((127 - sh) << 23);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            o[q] = pack_f16x2(__uint_as_float(wv[q] << 16) * down, __uint_as_float(wv[q] & 0xFFFF0000u) * down);
+          row[c ^ (frow & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
       }
       fence_proxy_async_smem();  // the converted row is read by the tensor cores
       __syncwarp();
@@ -670,6 +681,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       }
       const float2 ncc = make_float2(-c_run, -c_run);
       float2 zs2 = make_float2(0.f, 0.f);
+      float tm4[4] = {tmax, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
       const float4* nv = reinterpret_cast<const float4*>(nrm + s * 256);
       const float4* uv = reinterpret_cast<const float4*>(nrm + s * 256 + 128);
 #pragma unroll
@@ -682,21 +694,19 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
           const float* r = &ut[32 * q4 + 4 * k4];
           const float2 a01 = __ffma2_rn(make_float2(r[0], r[1]), make_float2(u4.x, u4.y), make_float2(n4.x, n4.y));
           const float2 a23 = __ffma2_rn(make_float2(r[2], r[3]), make_float2(u4.z, u4.w), make_float2(n4.z, n4.w));
-          tmax = max3(tmax, a01.x, a01.y);
-          tmax = max3(tmax, a23.x, a23.y);
+          tm4[k4 & 3] = max3(tm4[k4 & 3], a01.x, a01.y);
+          tm4[k4 & 3] = max3(tm4[k4 & 3], a23.x, a23.y);
           const float2 b01 = __fadd2_rn(a01, ncc), b23 = __fadd2_rn(a23, ncc);
           const float2 p01 = make_float2(ex2(b01.x), ex2(b01.y)), p23 = make_float2(ex2(b23.x), ex2(b23.y));
           zs2 = __fadd2_rn(zs2, __fadd2_rn(p01, p23));
           wph[2 * k4] = pack_bf16x2(p01.x, p01.y);
           wph[2 * k4 + 1] = pack_bf16x2(p23.x, p23.y);
         }
-        if (!fvalid) {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) wph[k] = 0u;
-        }
+        // (a feature past m has W' = 0; its S row is computed but never written out)
         tmem_st16(taddr(tbase, eq, cP + 16 * q4), wph);  // phi, bf16 pairs
       }
       zsum += zs2.x + zs2.y;
+      tmax = fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -760,10 +770,15 @@ struct QueryCfg {
   static constexpr int S_W = 0;                          // W' fp16, [D/64 regions][MMAX rows][128 B]
   static constexpr int S_SP = S_W + MMAX * 128 * (D / 64);
   static constexpr int S_Q = S_SP + SP;                  // Q stage w belongs to warpgroup w
-  static constexpr int S_STG = S_Q + 2 * QTILE;          // output staging, one 64-column region, shared
-  static constexpr int S_BAR = S_STG + 128 * 128;
+  // output staging, 32 rows x 64 columns per epilogue warp: a slot of its own at d = 64; at
+  // d = 128 (no room for eight) one slot per TMEM lane quarter, shared by the two warpgroups'
+  // warps of that quarter in tile order
+  static constexpr bool OWN_SLOT = D == 64;
+  static constexpr int NSLOT = OWN_SLOT ? 8 : 4;
+  static constexpr int S_STG = S_Q + 2 * QTILE;
+  static constexpr int S_BAR = S_STG + NSLOT * 32 * 128;
   static constexpr int B_QF = 0, B_QE = 2, B_CVT = 4, B_UF = 6, B_UE = 8, B_PHI = 10, B_M2 = 12, B_OF = 14,
-                       B_OE = 16, B_SF = 18, B_SE = 19, B_STG = 20, NBAR = 21;
+                       B_OE = 16, B_SF = 18, B_SE = 19, B_STG = 20, NBAR = 24;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int SMEM = S_ABORT + 16 + 1024;
@@ -829,7 +844,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     }
     mbar_init(bar(C::B_SF), 1);
     mbar_init(bar(C::B_SE), 2);  // an image is released once both issuers are done with it
-    mbar_init(bar(C::B_STG), 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(C::B_STG + i), 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmQ);
@@ -878,7 +893,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       int loaded = -1, issued = 0;
       for (int it = 0; it < n; ++it) {
         const int T = T0 + it, s = it & 1;
-        if (it >= 2 && !mbar_wait(bar(C::B_QE + s), ((it >> 1) - 1) & 1, abort_flag, err)) break;
+        if (it >= 2 && !mbar_wait<true>(bar(C::B_QE + s), ((it >> 1) - 1) & 1, abort_flag, err)) break;
         mbar_arrive_expect_tx(bar(C::B_QF + s), C::QTILE);
         const int bh = T / ntq, qt = T % ntq;
 #pragma unroll
@@ -994,40 +1009,47 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     const int eq = warp & 3;
     const int ewg = (warp - C::EPI0) >> 2;
     const int r = eq * 32 + lane;  // query row within the tile (TMEM lane)
-    const bool issuer = (eq == 0 && lane == 0);
     const uint32_t cU = ewg * C::TSTRIDE, cP = cU + FB, cO = cP + FB / 2;  // TMEM columns
     const int atoms = (m + 63) / 64;  // the image holds [atoms][D rows][64 features] fp16, then its tail
     const float* ev = reinterpret_cast<const float*>(smem + C::S_SP + D * 128 * atoms);
     const float* sd = ev + 64 * atoms;  // fp32 normaliser column of the state, same scaling as the image
-    // rewrites row r of Q tile t (Q stage ewg) as fp16 x 2^-k; returns 2^k.  Thread r starts at
-    // chunk r % 8 so that the eight threads of a shared-memory wavefront hit different banks.
+    // rewrites row r of Q tile t (Q stage ewg) as fp16 x 2^-k and returns 2^k; k = 0 unless the
+    // row's largest |q| reaches 2^15, when it brings it into [2^14, 2^15) so that no entry
+    // overflows fp16.  Thread r starts at chunk r % 8 so that the eight threads of a
+    // shared-memory wavefront hit different banks.
     auto prepare = [&](int tcount) -> float {
       mbar_wait(bar(C::B_QF + ewg), tcount & 1, abort_flag, err);
       unsigned char* qrow = smem + C::S_Q + ewg * C::QTILE + r * 128;
+      uint4 v[D / 8];
       uint32_t emax = 0;
 #pragma unroll
       for (int rg = 0; rg < D / 64; ++rg)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(qrow + rg * (128 * 128) + 16 * (c ^ (r & 7)));
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          v[8 * rg + c] = *reinterpret_cast<const uint4*>(qrow + rg * (128 * 128) + 16 * (c ^ (r & 7)));
+          const uint32_t wv[4] = {v[8 * rg + c].x, v[8 * rg + c].y, v[8 * rg + c].z, v[8 * rg + c].w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) emax = max(emax, max(wv[k] & 0x7F80u, (wv[k] >> 16) & 0x7F80u));
         }
-      const int k = min(100, max(-100, static_cast<int>(emax >> 7) - 141));
+      const int k = min(100, max(0, static_cast<int>(emax >> 7) - 141));
+      const bool plain = __all_sync(0xffffffffu, k == 0);
       const float down = __int_as_float((127 - k) << 23);
 #pragma unroll
       for (int rg = 0; rg < D / 64; ++rg)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          uint4* p = reinterpret_cast<uint4*>(qrow + rg * (128 * 128) + 16 * (c ^ (r & 7)));
-          const uint4 v = *p;
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          const uint32_t wv[4] = {v[8 * rg + c].x, v[8 * rg + c].y, v[8 * rg + c].z, v[8 * rg + c].w};
           uint32_t o[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            o[q] = pack_f16x2(__uint_as_float(wv[q] << 16) * down, __uint_as_float(wv[q] & 0xFFFF0000u) * down);
-          *p = make_uint4(o[0], o[1], o[2], o[3]);
+          for (int q = 0; q < 4; ++q) {
+            float lo = __uint_as_float(wv[q] << 16), hi = __uint_as_float(wv[q] & 0xFFFF0000u);
+            if (!plain) {
+              lo *= down;
+              hi *= down;
+            }
+            o[q] = pack_f16x2(lo, hi);
+          }
+          *reinterpret_cast<uint4*>(qrow + rg * (128 * 128) + 16 * (c ^ (r & 7))) = make_uint4(o[0], o[1], o[2], o[3]);
         }
       fence_proxy_async_smem();  // the converted tile is read by the tensor cores
       __syncwarp();
@@ -1086,7 +1108,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         if (need) c = mx;
         // phi' = 2^(2^k U + e - c) as fp16 pairs into the phi' buffer; normaliser in fp32
         const float2 nc2 = make_float2(-c, -c);
-        float2 den2 = make_float2(0.f, 0.f);
+        float2 den2 = make_float2(0.f, 0.f), den2b = make_float2(0.f, 0.f);  // two independent chains
 #pragma unroll
         for (int q4 = 0; q4 < FB / 32; ++q4) {
           uint32_t ph[16];
@@ -1097,13 +1119,13 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
             const float2 b01 = __fadd2_rn(make_float2(a[0], a[1]), nc2), b23 = __fadd2_rn(make_float2(a[2], a[3]), nc2);
             const float2 p01 = make_float2(ex2(b01.x), ex2(b01.y)), p23 = make_float2(ex2(b23.x), ex2(b23.y));
             den2 = __ffma2_rn(p01, make_float2(s4.x, s4.y), den2);
-            den2 = __ffma2_rn(p23, make_float2(s4.z, s4.w), den2);
+            den2b = __ffma2_rn(p23, make_float2(s4.z, s4.w), den2b);
             ph[2 * k4] = pack_f16x2(p01.x, p01.y);
             ph[2 * k4 + 1] = pack_f16x2(p23.x, p23.y);
           }
           tmem_st16(taddr(tbase, eq, cP + 16 * q4), ph);
         }
-        den += den2.x + den2.y;
+        den += (den2.x + den2.y) + (den2b.x + den2b.y);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -1115,13 +1137,19 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       mbar_wait(bar(C::B_OF + ewg), tc & 1, abort_flag, err);
       tc_fence_after();
       const float inv = 1.f / den;
-      if (t >= 1) mbar_wait(bar(C::B_STG), (t - 1) & 1, abort_flag, err);  // tile t - 1 released the staging tile
+      unsigned char* slot = smem + C::S_STG + ((C::OWN_SLOT ? 4 * ewg : 0) + eq) * (32 * 128);
+      if constexpr (C::OWN_SLOT) {  // this warp's previous store has read its slot
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      } else {  // the slot is free once the same quarter of tile t - 1 has been stored
+        if (t >= 1) mbar_wait(bar(C::B_STG + eq), (t - 1) & 1, abort_flag, err);
+      }
       const int T = T0 + t, bh = T / ntq, qt = T % ntq;
 #pragma unroll
       for (int rg = 0; rg < D / 64; ++rg) {
-        if (rg > 0) {
-          if (issuer) bulk_wait_read<0>();  // the previous region's store has read the staging tile
-          named_bar_sync(1 + ewg, 128);
+        if (rg > 0) {  // the previous region's store has read the slot
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
         }
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -1136,28 +1164,27 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
               w4[k] = pack_bf16x2(__uint_as_float(t32[8 * c4 + 2 * k]) * inv,
                                   __uint_as_float(t32[8 * c4 + 2 * k + 1]) * inv);
             const int c8 = 4 * h2 + c4;
-            *reinterpret_cast<uint4*>(smem + C::S_STG + r * 128 + ((c8 ^ (r & 7)) << 4)) =
-                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            *reinterpret_cast<uint4*>(slot + lane * 128 + ((c8 ^ (lane & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
-        if (rg == D / 64 - 1) {  // all of O has been read: the next tile may accumulate into it
+        if (rg == D / 64 - 1) {  // this warp has read all of its O rows: the next tile may accumulate
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(C::B_OE + ewg));
         }
         fence_proxy_async_smem();
-        named_bar_sync(1 + ewg, 128);
-        if (issuer) {
-          tma_store_3d(&tmO, sbase + C::S_STG, 64 * rg, qt * 128, bh);
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmO, smem_u32(slot), 64 * rg, qt * 128 + 32 * eq, bh);
           bulk_commit();
         }
       }
-      if (issuer) {
+      if (!C::OWN_SLOT && lane == 0) {
         bulk_wait_read<0>();
-        mbar_arrive(bar(C::B_STG));  // the staging tile is free for tile t + 1
+        mbar_arrive(bar(C::B_STG + eq));  // the slot is free for tile t + 1
       }
     }
-    if (issuer) bulk_wait<0>();
+    if (lane == 0) bulk_wait<0>();
   }
   tc_fence_before();
   __syncthreads();
@@ -1187,12 +1214,12 @@ EncodeTiledFn encode_fn() {
 
 // [heads, L, d] bf16, boxes of 64 dims x 128 rows x 1 head, 128-byte swizzle; rows past L read as zero
 // and are not written.
-int make_map(CUtensorMap* map, const void* base, int d, int L, int heads) {
+int make_map(CUtensorMap* map, const void* base, int d, int L, int heads, int box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return set_error(FAVOR_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(heads)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1255,7 +1282,7 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   CUtensorMap mq, mo;
   const int bh = p.B * p.H;
   int rc = make_map(&mq, Q, D, p.L, bh);
-  if (rc == FAVOR_OK) rc = make_map(&mo, out, D, p.L, bh);
+  if (rc == FAVOR_OK) rc = make_map(&mo, out, D, p.L, bh, 32);  // stored by each epilogue warp, 32 rows
   if (rc != FAVOR_OK) return rc;
   auto kern = query_pass_sm100<D>;
   static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), C::THREADS);
