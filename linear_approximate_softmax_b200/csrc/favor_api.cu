@@ -115,9 +115,10 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
   // the query pass's state operand: d rows of fp16 (the normaliser column goes to the tail)
   p->op_rows = d;
   p->op_atoms = (m + 63) / 64;
+  p->op_tail = (m + 127) / 128 * 128;
   // fp16 rows (64 features per 128-byte row), then one fp32 exponent per feature, then the
   // fp32 normaliser column with the same per-feature scaling
-  p->op_bytes = static_cast<size_t>(p->op_rows) * 128 * p->op_atoms + 512 * static_cast<size_t>(p->op_atoms);
+  p->op_bytes = static_cast<size_t>(p->op_rows) * 128 * p->op_atoms + 8 * static_cast<size_t>(p->op_tail);
   p->st_bytes = p->st_op_off + round_up(p->op_bytes * heads, 256);
   p->wscale = static_cast<float>(std::pow(static_cast<double>(d), -0.25) * kLog2e);
   p->nscale = static_cast<float>(std::pow(static_cast<double>(d), -0.5) * kLog2e * 0.5);

@@ -32,12 +32,14 @@ struct Plan {
   // byte offsets inside the state buffer
   size_t st_S_off, st_c_off, st_op_off, st_bytes;
   // The state re-packed as the fp16 B operand of the query pass's second MMA.
-  // Per kv head: op_atoms blocks of 64 features, each op_rows rows (output
-  // column n: d value columns, the normaliser at n = d, zeros after) of 128 B,
-  // K-major with the 128-byte swizzle (16-byte chunk c of row n at c ^ (n % 8));
-  // then e[64 * op_atoms] fp32.  Feature f's values are S[f][n] * 2^-e[f], with
-  // e[f] chosen so that the largest |S[f][n]| lands in [2^14, 2^15).
-  int op_rows, op_atoms;
+  // Per kv head: op_atoms blocks of 64 features, each op_rows = d rows (output
+  // column n) of 128 B, K-major with the 128-byte swizzle (16-byte chunk c of row n
+  // at c ^ (n % 8)); then e[op_tail] and the normaliser column s[op_tail], fp32, with
+  // op_tail = m rounded up to 128.  Feature f's values are 2^-x_f S[f][n] relative to
+  // its own largest chunk stabiliser c_f, with x_f chosen so that the largest lands in
+  // [2^14, 2^15); e[f] = x_f + c_f - c*, and e[f] = -inf for f >= m, so that the query
+  // pass needs no masking of the features past m.
+  int op_rows, op_atoms, op_tail;
   size_t op_bytes;
   float wscale;     // d^-1/4 * log2(e): W is multiplied by this on the device
   float nscale;     // d^-1/2 * log2(e) / 2: |k|^2 is multiplied by this

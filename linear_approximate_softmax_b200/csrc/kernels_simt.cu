@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads) key_pass_kernel(
   for (int f = tid; f < fbw; f += kThreads) part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + f] = c_run;
 }
 
-// grid (op_atoms * 64 / 32, B*Hkv), 256 threads: 32 feature rows per CTA, 8 threads
+// grid (op_tail / 32, B*Hkv), 256 threads: 32 feature rows per CTA, 8 threads
 // per row.  Each row is the sum of the chunk partials in the fixed order p = 0..P-1,
 // each rescaled from its own stabiliser to the row's largest one c_f (bitwise
 // deterministic).  Writes S[f][n] = 2^(c_f - c*) x that sum (fp32, relative to the head's
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kThreads) key_pass_kernel(
 __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
     const float* __restrict__ part_S, const float* __restrict__ part_c, float* __restrict__ S,
     float* __restrict__ Sc, unsigned char* __restrict__ op, int P, int m, int D1, int nsb, int op_rows,
-    int op_atoms, size_t op_bytes) {
+    int op_atoms, int op_tail, size_t op_bytes) {
   __shared__ float red[kThreads / 32];
   const int head = blockIdx.y;
   const float* pc = part_c + static_cast<size_t>(head) * P * nsb;
@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
 #pragma unroll
   for (int k = 0; k < kMaxCols; ++k) {
     const int n = g + 8 * k;
-    if (n < op_rows) {
+    if (n < op_rows && atom < op_atoms) {
       const size_t off = static_cast<size_t>(atom) * op_rows * 128 + static_cast<size_t>(n) * 128 +
                          ((chunk ^ (n & 7)) << 4) + el * 2;
       *reinterpret_cast<__half*>(img + off) = __float2half_rn(ldexpf(val[k], -ex));
@@ -230,8 +230,8 @@ __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
   }
   // tail: the exponent of each feature, then its normaliser entry with the same scaling
   float* tail = reinterpret_cast<float*>(img + static_cast<size_t>(op_rows) * 128 * op_atoms);
-  if (g == 0) tail[f] = live && cf > -INFINITY ? static_cast<float>(ex) + (cf - cs) : 0.f;
-  if (((D1 - 1) & 7) == g) tail[64 * op_atoms + f] = ldexpf(den, -ex);
+  if (g == 0) tail[f] = live && cf > -INFINITY ? static_cast<float>(ex) + (cf - cs) : -INFINITY;
+  if (((D1 - 1) & 7) == g) tail[op_tail + f] = live ? ldexpf(den, -ex) : 0.f;
 }
 
 // grid (ceil(L/32), B*H), 256 threads.
@@ -364,13 +364,14 @@ int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void*
 int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int D1 = p.d + 1;
-  dim3 grid(p.op_atoms * 64 / 32, p.B * p.Hkv);
+  dim3 grid(p.op_tail / 32, p.B * p.Hkv);
   const char* pb = static_cast<const char*>(partials);
   char* sb = static_cast<char*>(state);
   state_reduce_kernel<<<grid, kThreads, 0, st>>>(
       reinterpret_cast<const float*>(pb + p.part_S_off), reinterpret_cast<const float*>(pb + p.part_c_off),
       reinterpret_cast<float*>(sb + p.st_S_off), reinterpret_cast<float*>(sb + p.st_c_off),
-      reinterpret_cast<unsigned char*>(sb + p.st_op_off), p.P, p.m, D1, p.nsb, p.op_rows, p.op_atoms, p.op_bytes);
+      reinterpret_cast<unsigned char*>(sb + p.st_op_off), p.P, p.m, D1, p.nsb, p.op_rows, p.op_atoms, p.op_tail,
+      p.op_bytes);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "state reduce launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;

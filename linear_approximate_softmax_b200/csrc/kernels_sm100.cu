@@ -934,9 +934,11 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         ++rel;
         return true;
       };
-      auto mma1 = [&](int b) {  // U = (2^-k Q) W'^T in fp16 for my block b
-        const int j = b % nb, bw = min(FB, m - FB * j);
-        const uint32_t id1 = idesc_f16(128, bw, false, false);
+      // U = (2^-k Q) W'^T in fp16 for my block b, always FB columns wide: W' rows past m are
+      // zero, so every U column the epilogue reads is written (its e = -inf masks it)
+      const uint32_t id1 = idesc_f16(128, FB, false, false);
+      auto mma1 = [&](int b) {
+        const int j = b % nb;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
@@ -1010,9 +1012,11 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     const int ewg = (warp - C::EPI0) >> 2;
     const int r = eq * 32 + lane;  // query row within the tile (TMEM lane)
     const uint32_t cU = ewg * C::TSTRIDE, cP = cU + FB, cO = cP + FB / 2;  // TMEM columns
-    const int atoms = (m + 63) / 64;  // the image holds [atoms][D rows][64 features] fp16, then its tail
+    // the image holds [atoms][D rows][64 features] fp16, then e and the normaliser column (fp32,
+    // same scaling as the image), each over m rounded up to 128 features, e = -inf past m
+    const int atoms = (m + 63) / 64, tail = (m + 127) / 128 * 128;
     const float* ev = reinterpret_cast<const float*>(smem + C::S_SP + D * 128 * atoms);
-    const float* sd = ev + 64 * atoms;  // fp32 normaliser column of the state, same scaling as the image
+    const float* sd = ev + tail;
     // rewrites row r of Q tile t (Q stage ewg) as fp16 x 2^-k and returns 2^k; k = 0 unless the
     // row's largest |q| reaches 2^15, when it brings it into [2^14, 2^15) so that no entry
     // overflows fp16.  Thread r starts at chunk r % 8 so that the eight threads of a
@@ -1082,15 +1086,10 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
           const float4 e4 = e4p[k4];
           const float2 v01 = __ffma2_rn(make_float2(v[4 * k4 + 0], v[4 * k4 + 1]), up2, make_float2(e4.x, e4.y));
           const float2 v23 = __ffma2_rn(make_float2(v[4 * k4 + 2], v[4 * k4 + 3]), up2, make_float2(e4.z, e4.w));
-          v[4 * k4 + 0] = v01.x;
+          v[4 * k4 + 0] = v01.x;  // a feature past m has W' = 0 and e = -inf: v = -inf
           v[4 * k4 + 1] = v01.y;
           v[4 * k4 + 2] = v23.x;
           v[4 * k4 + 3] = v23.y;
-          if (FB * j + FB > m) {  // features past m (a warp-uniform condition)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (FB * j + 4 * k4 + e >= m) v[4 * k4 + e] = -INFINITY;
-          }
           m4[k4 & 3] = max3(m4[k4 & 3], v[4 * k4 + 0], v[4 * k4 + 1]);
           m4[k4 & 3] = max3(m4[k4 & 3], v[4 * k4 + 2], v[4 * k4 + 3]);
         }
