@@ -415,17 +415,18 @@ struct KeyPP {
   // warpgroups (each covers the four TMEM lane quarters once, as warp % 4)
   static constexpr int THREADS = 384;
   static constexpr int EPI0 = 4;
-  static constexpr int NST = 6;  // K/V stages: a tile is prepared two tiles ahead of its use
+  static constexpr int NST = 5;  // K/V stages: a tile's norms are taken two tiles ahead of its use
   static constexpr int TILE = 128 * 64 * 2;
   // TMEM columns: warpgroup w owns U^T at 256 w, phi at 256 w + 128 (bf16 pairs), S at 256 w + 192
   static constexpr int T_U = 0, T_P = 128, T_S = 192, T_STRIDE = 256;
-  static constexpr int S_W = 0;                     // W' fp16, 128 features x 64 dims, K-major SW128 (A of MMA1)
-  static constexpr int S_K = S_W + 128 * 128;
+  // W' = hi + lo in bf16, each 128 features x 64 dims, K-major SW128 (the A operands of MMA1)
+  static constexpr int S_WHI = 0, S_WLO = 128 * 128;
+  static constexpr int S_K = S_WLO + 128 * 128;
   static constexpr int S_V = S_K + NST * TILE;
-  static constexpr int S_NRM = S_V + NST * TILE;    // per stage: -n(k) [128], then 2^s [128]
-  static constexpr int S_CW = S_NRM + NST * 1024;   // final stabilisers and normalisers, [2][2][128]
+  static constexpr int S_NRM = S_V + NST * TILE;    // per stage: -n(k) [128]
+  static constexpr int S_CW = S_NRM + NST * 512;    // final stabilisers and normalisers, [2][2][128]
   static constexpr int S_BAR = S_CW + 2048;
-  static constexpr int B_KVF = 0, B_KVE = NST, B_CVT = 2 * NST, B_D1F = B_CVT + 2, B_UE = B_D1F + 2,
+  static constexpr int B_KVF = 0, B_KVE = NST, B_NRM = 2 * NST, B_D1F = B_NRM + 2, B_UE = B_D1F + 2,
                        B_PHI = B_UE + 2, B_SDONE = B_PHI + 2, NBAR = B_SDONE + 2;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
@@ -461,7 +462,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       mbar_init(bar(C::B_KVE + s), 1);
     }
     for (int w = 0; w < 2; ++w) {
-      mbar_init(bar(C::B_CVT + w), 4);  // one arrival per epilogue warp
+      mbar_init(bar(C::B_NRM + w), 4);  // one arrival per epilogue warp
       mbar_init(bar(C::B_D1F + w), 1);
       mbar_init(bar(C::B_UE + w), 4);
       mbar_init(bar(C::B_PHI + w), 4);
@@ -476,10 +477,12 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     tmem_alloc(smem_u32(tptr_slot), 512);
     tmem_relinquish();
   }
-  // W' fp16 as the K-major 128B-swizzled A operand of MMA1: row f, 16-byte chunk c at c ^ (f % 8)
+  // W' = hi + lo (bf16) as the K-major 128B-swizzled A operands of MMA1: row f, 16-byte chunk c
+  // at c ^ (f % 8); the pair keeps ~16 bits of W', so the exponents stay within the bf16
+  // output tolerance on heavy-tailed keys
   for (int item = tid; item < 128 * 8; item += C::THREADS) {
     const int f = item >> 3, c = item & 7;
-    uint32_t h[4];
+    uint32_t hi[4], lo[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       float w0 = 0.f, w1 = 0.f;
@@ -488,9 +491,12 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
         w0 = v.x * wscale;
         w1 = v.y * wscale;
       }
-      h[k] = pack_f16x2(w0, w1);
+      hi[k] = pack_bf16x2(w0, w1);
+      lo[k] = pack_bf16x2(w0 - __uint_as_float(hi[k] << 16), w1 - __uint_as_float(hi[k] & 0xFFFF0000u));
     }
-    *reinterpret_cast<uint4*>(smem + C::S_W + f * 128 + ((c ^ (f & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+    const int off = f * 128 + ((c ^ (f & 7)) << 4);
+    *reinterpret_cast<uint4*>(smem + C::S_WHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(smem + C::S_WLO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -526,20 +532,22 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     // U^T, ahead of this tile's contraction.
     if (lane == 0) {
       const int w = warp - 1;
-      const uint32_t id1 = idesc_f16(128, 128, false, false);
+      const uint32_t id1 = idesc_bf16(128, 128, false, false);
       const uint32_t idv = idesc_bf16(128, D, false, true);  // V tile as an MN-major B operand
       const uint32_t dU = tbase + w * C::T_STRIDE + C::T_U, dP = tbase + w * C::T_STRIDE + C::T_P,
                      dS = tbase + w * C::T_STRIDE + C::T_S;
-      auto mma1 = [&](int i) {  // U^T = W' (2^-s K)^T in fp16
+      auto mma1 = [&](int i) {  // U^T = (W'hi + W'lo) K^T
         const int s = i % C::NST;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          mma_ss(dU, sdesc_sw128(sbase + C::S_W + 32 * ks, 16, 1024),
-                 sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * ks, 16, 1024), id1, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < 2 * (D / 16); ++ks) {
+          const int kk = ks % (D / 16);
+          mma_ss(dU, sdesc_sw128(sbase + (ks < D / 16 ? C::S_WHI : C::S_WLO) + 32 * kk, 16, 1024),
+                 sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * kk, 16, 1024), id1, ks > 0 ? 1u : 0u);
+        }
         mma_commit(bar(C::B_D1F + w));
       };
       int cnt = 0;
-      bool ok = w < ntiles && mbar_wait(bar(C::B_CVT + w), 0, abort_flag, err);
+      bool ok = w < ntiles && mbar_wait(bar(C::B_KVF + w % C::NST), (w / C::NST) & 1, abort_flag, err);
       if (ok) {
         tc_fence_after();
         mma1(w);
@@ -547,8 +555,9 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       for (int i = w; i < ntiles && ok; i += 2, ++cnt) {
         const int s = i % C::NST;
         if (i + 2 < ntiles) {
-          if (!mbar_wait(bar(C::B_UE + w), cnt & 1, abort_flag, err)) break;         // U^T of tile i read
-          if (!mbar_wait(bar(C::B_CVT + w), (cnt + 1) & 1, abort_flag, err)) break;  // tile i + 2 prepared
+          if (!mbar_wait(bar(C::B_UE + w), cnt & 1, abort_flag, err)) break;  // U^T of tile i read
+          const int s2 = (i + 2) % C::NST;
+          if (!mbar_wait(bar(C::B_KVF + s2), ((i + 2) / C::NST) & 1, abort_flag, err)) break;  // tile i + 2 landed
           tc_fence_after();
           mma1(i + 2);
         }
@@ -596,60 +605,29 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     float c_run = floor_c, tmax = -INFINITY, zsum = 0.f;  // zsum: this feature's normaliser sum_t phi
     const uint32_t cU = ewg * C::T_STRIDE + C::T_U, cP = ewg * C::T_STRIDE + C::T_P,
                    cS = ewg * C::T_STRIDE + C::T_S;
-    // Prepares tile i for its projection, one key row (token frow) per thread: stores
-    // -n(k) = -|k|^2 nscale (-inf past the chunk end) and 2^s, and rewrites the bf16 row in
-    // place as fp16 times 2^-s.  s = 0 unless |k| >= 2^15, when it brings |k| 2^-s into
-    // [2^14, 2^15) so that no entry overflows fp16; an entry below fp16's normal range keeps an
-    // absolute error under 2^-25, which moves an exponent by less than |w'|_1 2^-25.  The
-    // 16-byte chunks of a swizzled row are summed in any order; thread frow starts at chunk
-    // frow % 8, so the eight threads of a shared-memory wavefront hit different banks.
+    // The key norms of tile i, one key row (token frow) per thread: -n(k) = -|k|^2 nscale
+    // (-inf past the chunk end), for the whole warpgroup once all four warps have arrived on
+    // B_NRM.  The 16-byte chunks of a swizzled row are summed in any order; thread frow starts
+    // at chunk frow % 8, so the eight threads of a shared-memory wavefront hit different banks.
     auto prepare_tile = [&](int i) {
       const int s = i % C::NST;
       mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err);
-      uint4* row = reinterpret_cast<uint4*>(smem + C::S_K + s * C::TILE + frow * 128);
-      uint4 v[8];
+      const uint4* row = reinterpret_cast<const uint4*>(smem + C::S_K + s * C::TILE + frow * 128);
       float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        v[c] = row[c ^ (frow & 7)];
-        const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+        const uint4 v = row[c ^ (frow & 7)];
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 x = make_float2(__uint_as_float(wv[k] << 16), __uint_as_float(wv[k] & 0xFFFF0000u));
-          acc[k & 1] = __ffma2_rn(x, x, acc[k & 1]);
+        for (int q = 0; q < 4; ++q) {
+          const float2 x = make_float2(__uint_as_float(wv[q] << 16), __uint_as_float(wv[q] & 0xFFFF0000u));
+          acc[q & 1] = __ffma2_rn(x, x, acc[q & 1]);
         }
       }
       const float sum = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
-      // |k| < 2^((E+1)/2) <= 2^(floor(E/2)+1) for sum = |k|^2 in [2^E, 2^(E+1))
-      const int e2 = static_cast<int>((__float_as_uint(sum) >> 23) & 0xFF) - 127;
-      const int sh = min(100, max(0, (e2 >> 1) + 1 - 15));
-      const bool inside = t_begin + 128 * i + frow < t_end;
-      nrm[s * 256 + frow] = inside ? -sum * nscale : -INFINITY;
-      nrm[s * 256 + 128 + frow] = __int_as_float((127 + sh) << 23);
-      if (__all_sync(0xffffffffu, sh == 0)) {  // the usual case: a plain conversion
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-          uint32_t o[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) o[q] = pack_f16x2(__uint_as_float(wv[q] << 16), __uint_as_float(wv[q] & 0xFFFF0000u));
-          row[c ^ (frow & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-      } else {
-        const float down = __int_as_float((127 - sh) << 23);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-          uint32_t o[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            o[q] = pack_f16x2(__uint_as_float(wv[q] << 16) * down, __uint_as_float(wv[q] & 0xFFFF0000u) * down);
-          row[c ^ (frow & 7)] = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-      }
-      fence_proxy_async_smem();  // the converted row is read by the tensor cores
+      nrm[s * 128 + frow] = (t_begin + 128 * i + frow < t_end) ? -sum * nscale : -INFINITY;
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_CVT + ewg));  // this warp's 32 rows are ready
+      if (lane == 0) mbar_arrive(bar(C::B_NRM + ewg));  // this warp's 32 norms are stored
     };
     int cnt = 0;
     if (ewg < ntiles) prepare_tile(ewg);
@@ -658,9 +636,9 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       mbar_wait(bar(C::B_D1F + ewg), cnt & 1, abort_flag, err);
       // every warp's norms of tile i are visible once all four have arrived for it (this
       // warp waits before arriving for tile i + 2, so the phase cannot have moved on)
-      mbar_wait(bar(C::B_CVT + ewg), cnt & 1, abort_flag, err);
-      // the projection of i + 2 is issued as soon as this tile's U^T has been read; preparing it
-      // only after U^T of i has arrived keeps each preparation one phase ahead of its consumer
+      mbar_wait(bar(C::B_NRM + ewg), cnt & 1, abort_flag, err);
+      // the norms of tile i + 2, two tiles ahead (after U^T of i has arrived, so that each
+      // warp's arrival stays one phase ahead of the waits on it)
       if (i + 2 < ntiles) prepare_tile(i + 2);
       // this tile's U^T row into registers (one read), then release it to the next projection
       float ut[128];
@@ -682,18 +660,16 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       const float2 ncc = make_float2(-c_run, -c_run);
       float2 zs2 = make_float2(0.f, 0.f);
       float tm4[4] = {tmax, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
-      const float4* nv = reinterpret_cast<const float4*>(nrm + s * 256);
-      const float4* uv = reinterpret_cast<const float4*>(nrm + s * 256 + 128);
+      const float4* nv = reinterpret_cast<const float4*>(nrm + s * 128);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t wph[16];
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {  // two tokens per packed fp32x2 operation
           const float4 n4 = nv[8 * q4 + k4];
-          const float4 u4 = uv[8 * q4 + k4];
           const float* r = &ut[32 * q4 + 4 * k4];
-          const float2 a01 = __ffma2_rn(make_float2(r[0], r[1]), make_float2(u4.x, u4.y), make_float2(n4.x, n4.y));
-          const float2 a23 = __ffma2_rn(make_float2(r[2], r[3]), make_float2(u4.z, u4.w), make_float2(n4.z, n4.w));
+          const float2 a01 = __fadd2_rn(make_float2(r[0], r[1]), make_float2(n4.x, n4.y));
+          const float2 a23 = __fadd2_rn(make_float2(r[2], r[3]), make_float2(n4.z, n4.w));
           tm4[k4 & 3] = max3(tm4[k4 & 3], a01.x, a01.y);
           tm4[k4 & 3] = max3(tm4[k4 & 3], a23.x, a23.y);
           const float2 b01 = __fadd2_rn(a01, ncc), b23 = __fadd2_rn(a23, ncc);
@@ -1033,9 +1009,11 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
           v[8 * rg + c] = *reinterpret_cast<const uint4*>(qrow + rg * (128 * 128) + 16 * (c ^ (r & 7)));
           const uint32_t wv[4] = {v[8 * rg + c].x, v[8 * rg + c].y, v[8 * rg + c].z, v[8 * rg + c].w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) emax = max(emax, max(wv[k] & 0x7F80u, (wv[k] >> 16) & 0x7F80u));
+          for (int k = 0; k < 4; ++k) emax = __vmaxu2(emax, wv[k] & 0x7FFF7FFFu);  // |q| of both halves
         }
-      const int k = min(100, max(0, static_cast<int>(emax >> 7) - 141));
+      // the biased bf16 exponent of the row's largest |q|
+      const int ebits = static_cast<int>(max(emax & 0xFFFFu, emax >> 16) >> 7);
+      const int k = min(100, max(0, ebits - 141));
       const bool plain = __all_sync(0xffffffffu, k == 0);
       const float down = __int_as_float((127 - k) << 23);
 #pragma unroll
