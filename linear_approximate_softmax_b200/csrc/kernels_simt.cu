@@ -188,15 +188,34 @@ __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
   if (live)
     for (int p = 0; p < P; ++p) cf = fmaxf(cf, pc[p * nsb + f / kStabBlock]);
   if (cf > -INFINITY) {
-    for (int p = 0; p < P; ++p) {
+    // chunks two at a time (both loads in flight), accumulated in the order p = 0..P-1
+    auto chunk_weight = [&](int p) {
       const float c = pc[p * nsb + f / kStabBlock];
-      if (c == -INFINITY) continue;
-      const float wp = exp2f(c - cf);
-      const float* src = part_S + ((static_cast<size_t>(head) * P + p) * m + f) * D1;
+      return c == -INFINITY ? 0.f : exp2f(c - cf);
+    };
+    auto chunk_row = [&](int p) { return part_S + ((static_cast<size_t>(head) * P + p) * m + f) * D1; };
+    int p = 0;
+    for (; p + 2 <= P; p += 2) {
+      const float w0 = chunk_weight(p), w1 = chunk_weight(p + 1);
+      const float* s0 = chunk_row(p);
+      const float* s1 = chunk_row(p + 1);
+      float x0[kMaxCols], x1[kMaxCols];
 #pragma unroll
       for (int k = 0; k < kMaxCols; ++k) {
         const int n = g + 8 * k;
-        if (n < D1) val[k] = fmaf(wp, src[n], val[k]);
+        x0[k] = n < D1 ? s0[n] : 0.f;
+        x1[k] = n < D1 ? s1[n] : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < kMaxCols; ++k) val[k] = fmaf(w1, x1[k], fmaf(w0, x0[k], val[k]));
+    }
+    if (p < P) {
+      const float w0 = chunk_weight(p);
+      const float* s0 = chunk_row(p);
+#pragma unroll
+      for (int k = 0; k < kMaxCols; ++k) {
+        const int n = g + 8 * k;
+        if (n < D1) val[k] = fmaf(w0, s0[n], val[k]);
       }
     }
   }
