@@ -700,7 +700,10 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     if (n1 > 0) mbar_wait(bar(C::B_SDONE + 1), (n1 - 1) & 1, abort_flag, err);
     tc_fence_after();
     const float s0 = n0 > 0 ? ex2(c0 - cmax) : 0.f, s1 = n1 > 0 ? ex2(c1 - cmax) : 0.f;
-    float* outp = part_S + (static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * (D + 1);
+    // the merged rows go through shared memory (the K stages are free now: every MMA has
+    // completed) so that the partial state is written with coalesced 16-byte stores; a row
+    // stride of D + 1 floats (odd) keeps the 32 rows of a warp on different banks
+    float* stg = reinterpret_cast<float*>(smem + C::S_K);
 #pragma unroll
     for (int cc = 0; cc < D / 16; ++cc) {  // this warpgroup's half of the columns
       const int col0 = ewg * (D / 2) + 8 * cc;
@@ -708,17 +711,20 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       tmem_ld8(taddr(tbase, eq, C::T_S + col0), v0);
       tmem_ld8(taddr(tbase, eq, C::T_STRIDE + C::T_S + col0), v1);
       tmem_wait_ld();
-      if (fvalid) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          outp[static_cast<size_t>(f0 + frow) * (D + 1) + col0 + k] =
-              fmaf(__uint_as_float(v1[k]), s1, __uint_as_float(v0[k]) * s0);
-      }
+      for (int k = 0; k < 8; ++k)
+        stg[frow * (D + 1) + col0 + k] = fmaf(__uint_as_float(v1[k]), s1, __uint_as_float(v0[k]) * s0);
     }
-    if (ewg == 0 && fvalid) {
-      outp[static_cast<size_t>(f0 + frow) * (D + 1) + D] = fmaf(cw[384 + frow], s1, cw[256 + frow] * s0);
-      part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + frow] = cmax;
+    if (ewg == 0) {
+      stg[frow * (D + 1) + D] = fmaf(cw[384 + frow], s1, cw[256 + frow] * s0);
+      if (fvalid) part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + frow] = cmax;
     }
+    named_bar_sync(3, 256);
+    // this group's rows f0 .. f0 + gw - 1 are contiguous in the partial state; gw (D + 1) is a
+    // multiple of 16 floats since m and f0 are multiples of 16
+    float4* outp = reinterpret_cast<float4*>(part_S + ((static_cast<size_t>(head) * P + p) * m + f0) * (D + 1));
+    const float4* src = reinterpret_cast<const float4*>(stg);
+    for (int i = tid - C::EPI0 * 32; i < gw * (D + 1) / 4; i += 256) outp[i] = src[i];
   }
   tc_fence_before();
   __syncthreads();
