@@ -56,6 +56,11 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}, "fallback"
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of each kernel on the
+# headline workload, from the ncu captures summarised in the named profiles/ files; a kernel
+# whose code changed after its capture gets no entry (traffic null).
+PROFILED_TRAFFIC = {}
+
 # MUFU ex2 issue rate of one B200 SM (16 results per clock) x 148 SMs x the
 # maximum SM clock: the exp roof of the path (derived from unit counts and clocks).
 MUFU_PER_SM_CLK = 16
@@ -312,7 +317,9 @@ def main():
                    "l2": f"inputs larger than L2 ({(Qh.numel() + Kh.numel() + Vh.numel()) * elt / 1e6:.0f} MB of Q,K,V per step)"},
         "roofline": {"kernel": names[dom], "bound": "alu", "achieved": achieved,
                      "peak": rt["mufu_peak_gexps"], "unit": "Gexp/s", "frac": achieved / rt["mufu_peak_gexps"],
-                     "traffic": None, "peak_source": f"MUFU 16/clk/SM x 148 SMs x {peaks['sm_max_mhz']:.0f} MHz"},
+                     "traffic": PROFILED_TRAFFIC.get((w.name, names[dom]), (None, None))[0],
+                     "traffic_source": PROFILED_TRAFFIC.get((w.name, names[dom]), (None, None))[1],
+                     "peak_source": f"MUFU 16/clk/SM x 148 SMs x {peaks['sm_max_mhz']:.0f} MHz"},
         "roofline_path": {"t_tensor_us": rt["t_tensor_us"], "t_mufu_us": rt["t_mufu_us"], "t_hbm_us": rt["t_hbm_us"],
                           "bound_us": max(rt["t_tensor_us"], rt["t_mufu_us"], rt["t_hbm_us"]),
                           "frac": max(rt["t_tensor_us"], rt["t_mufu_us"], rt["t_hbm_us"]) / (ms_per_step * 1e3),

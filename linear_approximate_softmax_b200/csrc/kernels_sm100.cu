@@ -472,6 +472,12 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     fence_barrier_init();
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    // the first stages' loads go out now, under the W' fill below
+    for (int i = 0; i < min(ntiles, C::NST); ++i) {
+      mbar_arrive_expect_tx(bar(C::B_KVF + i), 2 * C::TILE);
+      tma_load_3d(sbase + C::S_K + i * C::TILE, &tmK, bar(C::B_KVF + i), 0, t_begin + 128 * i, head);
+      tma_load_3d(sbase + C::S_V + i * C::TILE, &tmV, bar(C::B_KVF + i), 0, t_begin + 128 * i, head);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tptr_slot), 512);
@@ -513,10 +519,10 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
+      int issued = min(ntiles, C::NST);  // issued during the set-up
+      for (int i = issued; i < ntiles; ++i) {
         const int s = i % C::NST;
-        if (i >= C::NST && !mbar_wait<true>(bar(C::B_KVE + s), ((i / C::NST) - 1) & 1, abort_flag, err)) break;
+        if (!mbar_wait<true>(bar(C::B_KVE + s), ((i / C::NST) - 1) & 1, abort_flag, err)) break;
         mbar_arrive_expect_tx(bar(C::B_KVF + s), 2 * C::TILE);
         const int t0 = t_begin + 128 * i;
         tma_load_3d(sbase + C::S_K + s * C::TILE, &tmK, bar(C::B_KVF + s), 0, t0, head);
@@ -831,6 +837,19 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     fence_barrier_init();
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmO);
+    // the first two Q tiles and the first image go out now, under the W' fill below
+    for (int it = 0; it < min(n, 2); ++it) {
+      const int T = T0 + it;
+      mbar_arrive_expect_tx(bar(C::B_QF + it), C::QTILE);
+#pragma unroll
+      for (int r = 0; r < D / 64; ++r)
+        tma_load_3d(sbase + C::S_Q + it * C::QTILE + r * (128 * 128), &tmQ, bar(C::B_QF + it), 64 * r, (T % ntq) * 128,
+                    T / ntq);
+    }
+    if (n > 0) {
+      mbar_arrive_expect_tx(bar(C::B_SF), op_bytes);
+      bulk_load(sbase + C::S_SP, op_img + static_cast<size_t>(kvh0) * op_bytes, op_bytes, bar(C::B_SF));
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tptr_slot), 512);
@@ -872,15 +891,17 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   if (warp == 0) {
     // ---------------- producer: Q tiles (stage = tile parity) and state images ----------------
     if (lane == 0) {
-      int loaded = -1, issued = 0;
+      int loaded = n > 0 ? 0 : -1, issued = 0;  // tiles 0 and 1 and image 0 were issued during the set-up
       for (int it = 0; it < n; ++it) {
         const int T = T0 + it, s = it & 1;
-        if (it >= 2 && !mbar_wait<true>(bar(C::B_QE + s), ((it >> 1) - 1) & 1, abort_flag, err)) break;
-        mbar_arrive_expect_tx(bar(C::B_QF + s), C::QTILE);
-        const int bh = T / ntq, qt = T % ntq;
+        if (it >= 2) {
+          if (!mbar_wait<true>(bar(C::B_QE + s), ((it >> 1) - 1) & 1, abort_flag, err)) break;
+          mbar_arrive_expect_tx(bar(C::B_QF + s), C::QTILE);
+          const int bh = T / ntq, qt = T % ntq;
 #pragma unroll
-        for (int r = 0; r < D / 64; ++r)
-          tma_load_3d(sbase + C::S_Q + s * C::QTILE + r * (128 * 128), &tmQ, bar(C::B_QF + s), 64 * r, qt * 128, bh);
+          for (int r = 0; r < D / 64; ++r)
+            tma_load_3d(sbase + C::S_Q + s * C::QTILE + r * (128 * 128), &tmQ, bar(C::B_QF + s), 64 * r, qt * 128, bh);
+        }
         issued = it + 1;
         const int k = img(it);
         if (k > loaded) {  // a new kv head: load its image once both issuers have released the previous one
