@@ -59,7 +59,12 @@ def load_peaks():
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of each kernel on the
 # headline workload, from the ncu captures summarised in the named profiles/ files; a kernel
 # whose code changed after its capture gets no entry (traffic null).
-PROFILED_TRAFFIC = {}
+PROFILED_TRAFFIC = {
+    ("bf16_L16384_heavykeys", "query_pass"): (103.383040e6 + 57.270016e6,
+                                              "profiles/query_pass_sm100_bf16_L16384_heavykeys.md"),
+    ("bf16_L16384_heavykeys", "key_pass"): (201.481472e6 + 8.718848e6,
+                                            "profiles/key_pass_pp_sm100_bf16_L16384_heavykeys.md"),
+}
 
 # MUFU ex2 issue rate of one B200 SM (16 results per clock) x 148 SMs x the
 # maximum SM clock: the exp roof of the path (derived from unit counts and clocks).
