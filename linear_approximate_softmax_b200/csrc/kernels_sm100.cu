@@ -4,32 +4,30 @@
 // method): out = phi(Q')(phi(K')^T [V|1]) / last column, with positive random
 // features phi(x') = exp(W x' - |x'|^2/2)/sqrt(m).  Both contractions on each
 // side are dense, so they run on the tensor cores; the exp feature map (m
-// exponentials per token) runs on the MUFU between them.
+// exponentials per token) runs on the MUFU between them.  Everything is in log2
+// units: W' = d^-1/4 log2(e) W, n(k) = d^-1/2 log2(e) |k|^2 / 2.
 //
-// Key pass (one CTA per 128-feature group x key chunk x kv head), transposed:
-//   MMA1  U^T[f, t] = W'[f, :] . K[t, :]      A = W' (hi + lo bf16) in TMEM,  B = K tile (TMA, smem)
-//   exp   phi^T[f, t] = 2^(U^T - n(k_t) - c)  written back over U^T as bf16 (A operand of MMA2)
-//   MMA2  S[f, :] += phi^T[f, :] . [V | 1]    A = phi^T in TMEM, B = V tile (smem, MN-major) and a ones tile
-// so every thread of the two epilogue warpgroups owns one feature (TMEM lane)
-// and half of the tile's tokens.  c is the chunk's running max exponent, raised
-// only when a tile exceeds it by more than 2^8 (the accumulator is then rescaled
-// exactly); the state reduction later brings all chunks to one constant.
+// Key pass, d = 64 (one CTA per 128-feature group x key chunk x kv head; two
+// epilogue warpgroups on alternate 128-token tiles, each with its own MMA issuer):
+//   MMA1  U^T[f, t] = (W'hi + W'lo)[f, :] . K[t, :]   A = W' halves (smem), B = K tile (TMA)
+//   exp   phi^T[f, t] = 2^(U^T - n(k_t) - c_f)        bf16, into its own TMEM buffer
+//   MMA2  S[f, :] += phi^T[f, :] . V                  A = phi^T (TMEM), B = V tile (MN-major)
+// so every epilogue thread owns one feature (TMEM lane) and reads its U^T row once.
+// c_f is the feature's running max exponent, raised only when a tile exceeds it by
+// more than 2^8 (S and the normaliser sum are then rescaled exactly); the state
+// reduction brings all chunks to one constant per feature.
+// Key pass, d = 128: the lock-step variant (both warpgroups on each tile, W' hi + lo
+// in TMEM as the A operand, one N = d + 16 MMA2 against [V | ones]).
 //
-// Query pass (one CTA per SM over a contiguous range of 128-query tiles):
-//   MMA1  U[q, f] = Q[q, :] . W'[f, :]        A = Q tile (TMA), B = W' hi + lo (smem), per 128-feature block
-//   exp   phi'[q, f] = 2^(U + e_f - c_q)      fp16, written back over U; c_q = the row max of U + e,
-//                                             raised lazily across feature blocks
-//   MMA2  O[q, :] += phi'[q, block] . S'[block, :]   kind::f16: A = phi' in TMEM, B = fp16 state image
-//   out = O[:, :d] / O[:, d] -> bf16 -> TMA store.
-// The state image holds each feature row scaled by its own power of two, S' = 2^-e_f S,
-// so that fp16 keeps 11 bits for every row; adding e_f to the exponent restores the
-// product exactly.  bf16 operands (8 bits) cost up to 2^-8 of an output when one
-// feature dominates a query, which, with the bf16 output rounding, reaches the 2e-2
-// max-abs bound; tf32 would need twice the MMA instructions.
-//
-// W' = d^-1/4 log2(e) W is split as W' = hi + lo in bf16 so that the exponent
-// arguments keep ~17 bits: a single bf16 W' moves the exponents by up to
-// 2^-9 |W'x|, which fails the bf16 output tolerance on heavy-tailed keys.
+// Query pass (one persistent CTA per SM over a contiguous range of 128-query tiles;
+// two epilogue warpgroups on alternate tiles, each with its own MMA issuer):
+//   MMA1  U[q, f] = (2^-k_q Q)[q, :] . W'[f, :]       fp16, per block of FB features
+//   exp   phi'[q, f] = 2^(2^k_q U + e_f - c_q)         fp16, into its own TMEM buffer;
+//                                                       c_q = the row max, raised lazily
+//   MMA2  O[q, :] += phi'[q, block] . S'[block, :]      A = phi' (TMEM), B = fp16 state image
+//   out = O / (phi' . s) -> bf16 -> TMA store.
+// The state image holds each feature row scaled by its own power of two, so that fp16
+// keeps 11 bits for every row; adding e_f to the exponent restores the product.
 //
 // Every mbarrier wait is bounded (2 s); a CTA that gives up raises the device
 // error word, stops issuing work, drains its own copies and frees its TMEM.
@@ -77,7 +75,7 @@ __device__ __noinline__ void scale_tmem_row(uint32_t taddr0, int chunks, float s
 }
 
 // ============================================================================
-// Key pass
+// Key pass, d = 128: lock-step (both epilogue warpgroups on every tile)
 // ============================================================================
 template <int D>
 struct KeyCfg {
@@ -1261,12 +1259,19 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   int rc = make_map(&mk, K, D, p.L, heads);
   if (rc == FAVOR_OK) rc = make_map(&mv, V, D, p.L, heads);
   if (rc != FAVOR_OK) return rc;
-  auto kern = (D == 64) ? key_pass_pp_sm100 : key_pass_sm100<D>;
-  const int smem_bytes = (D == 64) ? KeyPP::SMEM : KeyCfg<D>::SMEM;
-  const int threads = (D == 64) ? KeyPP::THREADS : kThreads;
-  if (D == 64) {
+  // d = 64: the two-warpgroup kernel; d = 128: the lock-step kernel
+  void (*kern)(const CUtensorMap, const CUtensorMap, const float*, float*, float*, int, int, int, int, int, float, float);
+  int smem_bytes, threads;
+  if constexpr (D == 64) {
+    kern = key_pass_pp_sm100;
+    smem_bytes = KeyPP::SMEM;
+    threads = KeyPP::THREADS;
     static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), threads);
     if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), threads);
+  } else {
+    kern = key_pass_sm100<D>;
+    smem_bytes = KeyCfg<D>::SMEM;
+    threads = kThreads;
   }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass attribute: %s", cudaGetErrorString(e));

@@ -65,20 +65,6 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
   return ok != 0;
 }
 
-// Non-blocking probe of the same condition (mbarrier.test_wait never suspends the thread,
-// unlike try_wait): for a thread that polls several barriers in turn.
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Waits for the phase of `bar` with parity `parity` to complete.  Gives up after
 // `limit_ns` of wall time, or at once when *abort is set; on giving up it sets
 // *abort and the global error word and returns false.  Every pipeline wait in
@@ -100,28 +86,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       }
     }
   }
-}
-
-// Bookkeeping for a thread that polls several barriers with mbar_test: after a pass
-// that made no progress, counts it, and every 1024 such passes checks the SM clock;
-// gives up (setting *abort and the error word) after about 2^32 cycles (2-3 s) without
-// progress.  Reading a clock on every pass would cost more than the pass itself.
-__device__ __forceinline__ bool idle_poll(bool progressed, uint32_t& polls, long long& idle_since,
-                                          volatile int* abort, unsigned int* err_word) {
-  if (progressed) {
-    polls = 0;
-    return false;
-  }
-  if (polls == 0) idle_since = clock64();
-  if ((++polls & 1023u) == 0) {
-    if (*abort) return true;
-    if (clock64() - idle_since > (1ll << 32)) {
-      *abort = 1;
-      atomicOr(err_word, FAVOR_DEVERR_TIMEOUT);
-      return true;
-    }
-  }
-  return false;
 }
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
