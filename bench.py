@@ -72,6 +72,19 @@ MUFU_PER_SM_CLK = 16
 NUM_SMS = 148
 
 
+def max_over_ranks(x, dist):
+    """The largest of a per-rank float64 tensor over all ranks (in place), as a float."""
+    if dist:
+        import torch.distributed as td
+        td.all_reduce(x, op=td.ReduceOp.MAX)
+    return float(x.item())
+
+
+def whole_job_rate(units_per_rank, world, ms_per_step):
+    """Mtoken*heads/s of the whole job: every rank runs its own replica of the workload."""
+    return units_per_rank * world / (ms_per_step * 1e-3) / 1e6
+
+
 def roofline_terms(w, peaks):
     """Algorithmic work per step and the time each resource needs for it at peak."""
     G = w.H // w.Hkv
@@ -281,11 +294,8 @@ def main():
         td.barrier()
     ms_total = start.elapsed_time(stop)
     stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / steps for j in range(3)]
-    ms = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-    if dist:
-        td.all_reduce(ms, op=td.ReduceOp.MAX)
-    ms_per_step = float(ms.item()) / steps
-    value = w.units * world / (ms_per_step * 1e-3) / 1e6
+    ms_per_step = max_over_ranks(torch.tensor([ms_total], device=dev, dtype=torch.float64), dist) / steps
+    value = whole_job_rate(w.units, world, ms_per_step)
 
     # end to end through the host-buffer C-ABI call (pinned host memory)
     Qp, Kp, Vp, Op = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory(), torch.empty_like(Qh).pin_memory()
@@ -298,10 +308,8 @@ def main():
         fv.favor_attention_host(Qp, Kp, Vp, Wh, Op, stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], device=dev, dtype=torch.float64)
-    if dist:
-        td.all_reduce(e2e_ms, op=td.ReduceOp.MAX)
-    e2e_value = w.units * world / (float(e2e_ms.item()) * 1e-3) / 1e6
+    e2e_ms = max_over_ranks(torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], device=dev, dtype=torch.float64), dist)
+    e2e_value = whole_job_rate(w.units, world, e2e_ms)
     elt = Qh.element_size()
     h2d = (Qh.numel() + Kh.numel() + Vh.numel()) * elt + Wh.numel() * 4
     d2h = Qh.numel() * elt
@@ -331,7 +339,7 @@ def main():
                           "peaks": f"{peak_src}: HBM {peaks['hbm_gbs']} GB/s, bf16 {peaks['bf16_tflops']} TFLOP/s"},
         "stage_ms": dict(zip(names, stage_ms)),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": float(e2e_ms.item())},
+                "ms_per_step": e2e_ms},
         "gpu_launches": 3 * steps,
         "clocks": clocks.summary(),
     }
