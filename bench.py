@@ -277,8 +277,8 @@ def main():
         per = (time.perf_counter() - t) / 5
         steps = int(min(5000, max(20, 3.0 / max(per, 1e-6))))
 
-    # per-stage events on the launching stream, every step of the timed region
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    # the timed region: plain steps, so that each kernel's set-up overlaps the end of the one
+    # before it (events between the kernels would serialise them)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         import torch.distributed as td
@@ -287,13 +287,20 @@ def main():
     with ClockSampler(local) as clocks:
         start.record(stream)
         for i in range(steps):
-            step(evs[i])
+            step()
         stop.record(stream)
         torch.cuda.synchronize(dev)
     if dist:
         td.barrier()
     ms_total = start.elapsed_time(stop)
-    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / steps for j in range(3)]
+    # each kernel's own duration: events on the launching stream between the stages, in
+    # separate steps after the timed region
+    nst = min(steps, 50)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nst)]
+    for i in range(nst):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    stage_ms = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / nst for j in range(3)]
     ms_per_step = max_over_ranks(torch.tensor([ms_total], device=dev, dtype=torch.float64), dist) / steps
     value = whole_job_rate(w.units, world, ms_per_step)
 

@@ -24,6 +24,7 @@
 #include <cmath>
 
 #include "favor_internal.h"
+#include "launch.cuh"
 
 namespace favor {
 namespace {
@@ -160,73 +161,75 @@ __global__ void __launch_bounds__(kThreads) key_pass_kernel(
 // e_f = x_f + (c_f - c*) and the normaliser entry with the same scaling.  Because the
 // image carries c_f - c* in e_f rather than in its fp16 values, a feature whose keys sit
 // far below the head's largest exponent keeps its precision on the query side.
-__global__ void __launch_bounds__(kThreads) state_reduce_kernel(
+// The kernel is latency-bound: the rows of CB chunks, the feature's stabilisers and the
+// head's stabilisers are all requested before any of them is used, and the image goes out
+// through shared memory as whole 16-byte pieces of its rows.
+template <int D>
+__global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel(
     const float* __restrict__ part_S, const float* __restrict__ part_c, float* __restrict__ S,
-    float* __restrict__ Sc, unsigned char* __restrict__ op, int P, int m, int D1, int nsb, int op_rows,
-    int op_atoms, int op_tail, size_t op_bytes) {
+    float* __restrict__ Sc, unsigned char* __restrict__ op, int P, int m, int nsb, int op_atoms, int op_tail,
+    size_t op_bytes) {
+  constexpr int D1 = D + 1;
+  constexpr int NC = (D1 + 7) / 8;     // columns per thread: g, g + 8, ...
+  constexpr int CB = D == 64 ? 3 : 2;  // chunks whose rows are in flight together
   __shared__ float red[kThreads / 32];
-  const int head = blockIdx.y;
+  __shared__ __align__(16) __half stage[D][32];  // the image rows of this CTA's 32 features
+  griddep_launch_dependents();
+  griddep_wait();  // the partial state comes from the kernel before this one on the stream
+  const int head = blockIdx.y, tid = threadIdx.x;
+  const int fl = tid >> 3, f0 = blockIdx.x * 32, f = f0 + fl;  // feature row (< op_tail)
+  const int g = tid & 7;
+  const bool live = f < m;
   const float* pc = part_c + static_cast<size_t>(head) * P * nsb;
+  const float* rows = part_S + (static_cast<size_t>(head) * P * m + f) * D1;  // chunk p at + p * m * D1
+  float x[CB][NC];
+  auto load = [&](int p0) {
+#pragma unroll
+    for (int b = 0; b < CB; ++b)
+#pragma unroll
+      for (int k = 0; k < NC; ++k) {
+        const int n = g + 8 * k;
+        x[b][k] = live && p0 + b < P && n < D1 ? rows[static_cast<size_t>(p0 + b) * m * D1 + n] : 0.f;
+      }
+  };
+  load(0);
+  float cf = -INFINITY;  // this feature's largest chunk stabiliser
+  if (live)
+    for (int p = 0; p < P; ++p) cf = fmaxf(cf, pc[p * nsb + f / kStabBlock]);
   float cs = -INFINITY;  // the head's largest stabiliser
-  for (int i = threadIdx.x; i < P * nsb; i += kThreads) cs = fmaxf(cs, pc[i]);
+  for (int i = tid; i < P * nsb; i += kThreads) cs = fmaxf(cs, pc[i]);
+  float val[NC];
+#pragma unroll
+  for (int k = 0; k < NC; ++k) val[k] = 0.f;
+  for (int p0 = 0; p0 < P; p0 += CB) {
+    if (p0 > 0) load(p0);
+#pragma unroll
+    for (int b = 0; b < CB; ++b) {
+      const int p = p0 + b;
+      if (live && p < P) {
+        const float c = pc[p * nsb + f / kStabBlock];
+        const float w = c == -INFINITY ? 0.f : exp2f(c - cf);
+#pragma unroll
+        for (int k = 0; k < NC; ++k) val[k] = fmaf(w, x[b][k], val[k]);
+      }
+    }
+  }
   cs = warp_max(cs);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = cs;
+  if ((tid & 31) == 0) red[tid >> 5] = cs;
   __syncthreads();
   cs = red[0];
 #pragma unroll
   for (int w = 1; w < kThreads / 32; ++w) cs = fmaxf(cs, red[w]);
-  if (blockIdx.x == 0 && threadIdx.x == 0) Sc[head] = cs;
+  if (blockIdx.x == 0 && tid == 0) Sc[head] = cs;
 
-  const int f = blockIdx.x * 32 + (threadIdx.x >> 3);  // feature row (< op_atoms * 64)
-  const int g = threadIdx.x & 7;                       // this thread's columns: g, g + 8, ...
-  const bool live = f < m;
-  constexpr int kMaxCols = (128 + 16) / 8;             // max(op_rows, D1) <= 144
-  float val[kMaxCols];
-#pragma unroll
-  for (int k = 0; k < kMaxCols; ++k) val[k] = 0.f;
-  float cf = -INFINITY;  // this feature's largest chunk stabiliser
-  if (live)
-    for (int p = 0; p < P; ++p) cf = fmaxf(cf, pc[p * nsb + f / kStabBlock]);
-  if (cf > -INFINITY) {
-    // chunks two at a time (both loads in flight), accumulated in the order p = 0..P-1
-    auto chunk_weight = [&](int p) {
-      const float c = pc[p * nsb + f / kStabBlock];
-      return c == -INFINITY ? 0.f : exp2f(c - cf);
-    };
-    auto chunk_row = [&](int p) { return part_S + ((static_cast<size_t>(head) * P + p) * m + f) * D1; };
-    int p = 0;
-    for (; p + 2 <= P; p += 2) {
-      const float w0 = chunk_weight(p), w1 = chunk_weight(p + 1);
-      const float* s0 = chunk_row(p);
-      const float* s1 = chunk_row(p + 1);
-      float x0[kMaxCols], x1[kMaxCols];
-#pragma unroll
-      for (int k = 0; k < kMaxCols; ++k) {
-        const int n = g + 8 * k;
-        x0[k] = n < D1 ? s0[n] : 0.f;
-        x1[k] = n < D1 ? s1[n] : 0.f;
-      }
-#pragma unroll
-      for (int k = 0; k < kMaxCols; ++k) val[k] = fmaf(w1, x1[k], fmaf(w0, x0[k], val[k]));
-    }
-    if (p < P) {
-      const float w0 = chunk_weight(p);
-      const float* s0 = chunk_row(p);
-#pragma unroll
-      for (int k = 0; k < kMaxCols; ++k) {
-        const int n = g + 8 * k;
-        if (n < D1) val[k] = fmaf(w0, s0[n], val[k]);
-      }
-    }
-  }
   const float rel = cf > -INFINITY ? exp2f(cf - cs) : 0.f;  // the row relative to c*
   float amax = 0.f, den = 0.f;
 #pragma unroll
-  for (int k = 0; k < kMaxCols; ++k) {
+  for (int k = 0; k < NC; ++k) {
     const int n = g + 8 * k;
     if (live && n < D1) S[(static_cast<size_t>(head) * m + f) * D1 + n] = val[k] * rel;
-    if (n < op_rows) amax = fmaxf(amax, fabsf(val[k]));
-    if (n == D1 - 1) den = val[k];
+    if (n < D) amax = fmaxf(amax, fabsf(val[k]));
+    if (n == D) den = val[k];
   }
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
@@ -236,21 +239,26 @@ __global__ void __launch_bounds__(kThreads) state_reduce_kernel(
     frexpf(amax, &ex);  // amax = mant * 2^ex, mant in [0.5, 1)
     ex -= 15;           // amax * 2^-ex in [2^14, 2^15)
   }
-  unsigned char* img = op + static_cast<size_t>(head) * op_bytes;
-  const int atom = f >> 6, chunk = (f & 63) >> 3, el = f & 7;
 #pragma unroll
-  for (int k = 0; k < kMaxCols; ++k) {
+  for (int k = 0; k < NC; ++k) {
     const int n = g + 8 * k;
-    if (n < op_rows && atom < op_atoms) {
-      const size_t off = static_cast<size_t>(atom) * op_rows * 128 + static_cast<size_t>(n) * 128 +
-                         ((chunk ^ (n & 7)) << 4) + el * 2;
-      *reinterpret_cast<__half*>(img + off) = __float2half_rn(ldexpf(val[k], -ex));
-    }
+    if (n < D) stage[n][fl] = __float2half_rn(ldexpf(val[k], -ex));
   }
+  unsigned char* img = op + static_cast<size_t>(head) * op_bytes;
   // tail: the exponent of each feature, then its normaliser entry with the same scaling
-  float* tail = reinterpret_cast<float*>(img + static_cast<size_t>(op_rows) * 128 * op_atoms);
+  float* tail = reinterpret_cast<float*>(img + static_cast<size_t>(D) * 128 * op_atoms);
   if (g == 0) tail[f] = live && cf > -INFINITY ? static_cast<float>(ex) + (cf - cs) : -INFINITY;
-  if (((D1 - 1) & 7) == g) tail[op_tail + f] = live ? ldexpf(den, -ex) : 0.f;
+  if ((D & 7) == g) tail[op_tail + f] = live ? ldexpf(den, -ex) : 0.f;
+  __syncthreads();
+  // the image holds 64 features per 128-byte row (dimension n), 16-byte chunk c at c ^ (n % 8):
+  // this CTA's 32 features are four chunks of each row of its 64-feature atom
+  const int atom = f0 >> 6;
+  if (atom < op_atoms)
+    for (int i = tid; i < D * 4; i += kThreads) {
+      const int n = i >> 2, c4 = i & 3, chunk = ((f0 & 63) >> 3) + c4;
+      const size_t off = static_cast<size_t>(atom) * D * 128 + static_cast<size_t>(n) * 128 + ((chunk ^ (n & 7)) << 4);
+      *reinterpret_cast<uint4*>(img + off) = *reinterpret_cast<const uint4*>(&stage[n][8 * c4]);
+    }
 }
 
 // grid (ceil(L/32), B*H), 256 threads.
@@ -382,16 +390,15 @@ int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void*
 
 int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int D1 = p.d + 1;
   dim3 grid(p.op_tail / 32, p.B * p.Hkv);
   const char* pb = static_cast<const char*>(partials);
   char* sb = static_cast<char*>(state);
-  state_reduce_kernel<<<grid, kThreads, 0, st>>>(
-      reinterpret_cast<const float*>(pb + p.part_S_off), reinterpret_cast<const float*>(pb + p.part_c_off),
-      reinterpret_cast<float*>(sb + p.st_S_off), reinterpret_cast<float*>(sb + p.st_c_off),
-      reinterpret_cast<unsigned char*>(sb + p.st_op_off), p.P, p.m, D1, p.nsb, p.op_rows, p.op_atoms, p.op_tail,
-      p.op_bytes);
-  cudaError_t e = cudaGetLastError();
+  auto kern = p.d == 64 ? state_reduce_kernel<64> : state_reduce_kernel<128>;
+  cudaError_t e = launch_overlapped(
+      kern, grid, dim3(kThreads), 0, st, reinterpret_cast<const float*>(pb + p.part_S_off),
+      reinterpret_cast<const float*>(pb + p.part_c_off), reinterpret_cast<float*>(sb + p.st_S_off),
+      reinterpret_cast<float*>(sb + p.st_c_off), reinterpret_cast<unsigned char*>(sb + p.st_op_off), p.P, p.m, p.nsb,
+      p.op_atoms, p.op_tail, p.op_bytes);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "state reduce launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
 }

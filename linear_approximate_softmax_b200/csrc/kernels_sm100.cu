@@ -39,6 +39,7 @@
 #include <mutex>
 
 #include "favor_internal.h"
+#include "launch.cuh"
 #include "sm100_ptx.cuh"
 
 namespace favor {
@@ -112,6 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
     float nscale) {
   using C = KeyCfg<D>;
   extern __shared__ unsigned char smem_raw[];
+  griddep_launch_dependents();  // the next kernel on the stream may be scheduled as SMs free up
   // offset the __shared__ array itself (not via an integer cast), so that every pointer derived
   // from it stays a shared-memory pointer and compiles to shared loads and stores
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -371,7 +373,9 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_PHI + b));
     }
-    // state readout: S rows of this group -> partial [m][D+1]
+    // state readout: S rows of this group -> partial [m][D+1], once the kernels before this
+    // one on the stream (which may read the partial state) have completed
+    griddep_wait();
     mbar_wait(bar(C::B_SDONE), (ntiles - 1) & 1, abort_flag, err);
     tc_fence_after();
     float* outp = part_S + (static_cast<size_t>(head) * P + p) * static_cast<size_t>(m) * (D + 1);
@@ -439,6 +443,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
   using C = KeyPP;
   constexpr int D = C::D;
   extern __shared__ unsigned char smem_raw[];
+  griddep_launch_dependents();  // the next kernel on the stream may be scheduled as SMs free up
   // offset the __shared__ array itself (not via an integer cast), so that every pointer derived
   // from it stays a shared-memory pointer and compiles to shared loads and stores
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -693,7 +698,9 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       if (lane == 0) mbar_arrive(bar(C::B_PHI + ewg));
     }
     if (!fvalid) zsum = 0.f;
-    // merge the two accumulators row by row and write this group's partial state
+    // merge the two accumulators row by row and write this group's partial state, once the
+    // kernels before this one on the stream (which may read the partial state) have completed
+    griddep_wait();
     cw[ewg * 128 + frow] = c_run;
     cw[256 + ewg * 128 + frow] = zsum;
     named_bar_sync(3, 256);
@@ -792,6 +799,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   constexpr int NT = C::THREADS;
   constexpr int FB = C::FB;
   extern __shared__ unsigned char smem_raw[];
+  griddep_launch_dependents();  // the next kernel on the stream may be scheduled as SMs free up
   // offset the __shared__ array itself (not via an integer cast), so that every pointer derived
   // from it stays a shared-memory pointer and compiles to shared loads and stores
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -844,6 +852,8 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         tma_load_3d(sbase + C::S_Q + it * C::QTILE + r * (128 * 128), &tmQ, bar(C::B_QF + it), 64 * r, (T % ntq) * 128,
                     T / ntq);
     }
+    // the state images are written by the kernel before this one on the stream
+    griddep_wait();
     if (n > 0) {
       mbar_arrive_expect_tx(bar(C::B_SF), op_bytes);
       bulk_load(sbase + C::S_SP, op_img + static_cast<size_t>(kvh0) * op_bytes, op_bytes, bar(C::B_SF));
@@ -1277,10 +1287,9 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass attribute: %s", cudaGetErrorString(e));
   char* base = static_cast<char*>(partials);
   dim3 grid((p.m + 127) / 128, p.P, heads);
-  kern<<<grid, threads, smem_bytes, st>>>(mk, mv, W, reinterpret_cast<float*>(base + p.part_S_off),
-                                        reinterpret_cast<float*>(base + p.part_c_off), p.L, p.m, p.P, p.chunk,
-                                        p.nsb, p.wscale, p.nscale);
-  e = cudaGetLastError();
+  e = launch_overlapped(kern, grid, dim3(threads), smem_bytes, st, mk, mv, W,
+                        reinterpret_cast<float*>(base + p.part_S_off), reinterpret_cast<float*>(base + p.part_c_off),
+                        p.L, p.m, p.P, p.chunk, p.nsb, p.wscale, p.nscale);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
 }
@@ -1301,9 +1310,8 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   const int ntiles = bh * ((p.L + 127) / 128);
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
   const unsigned char* img = static_cast<const unsigned char*>(state) + p.st_op_off;
-  kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mo, W, img, p.L, p.m, p.H, p.Hkv, ntiles, static_cast<int>(p.op_bytes),
-                                        p.wscale);
-  e = cudaGetLastError();
+  e = launch_overlapped(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, mq, mo, W, img, p.L, p.m, p.H, p.Hkv,
+                        ntiles, static_cast<int>(p.op_bytes), p.wscale);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
 }
