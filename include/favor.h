@@ -123,10 +123,16 @@ FAVOR_API int favor_attention_f32(const float* Q, const float* K, const float* V
  *
  * Q, K, V, out are host pointers (pinned memory gives asynchronous copies;
  * pageable memory works, slower); W is a host [m,d] fp32 array.  dtype is
- * FAVOR_BF16 or FAVOR_F32 for Q, K, V and out.  The call copies the inputs to
- * the device, runs favor_attention(_f32) on `stream`, copies out back, and
- * synchronises `stream` before returning.  Device buffers are allocated and
- * freed stream-ordered inside the call.
+ * FAVOR_BF16 or FAVOR_F32 for Q, K, V and out.  The call splits the B*Hkv kv
+ * heads into at most 8 pieces of consecutive kv heads (each with its H/Hkv
+ * query heads, one contiguous range of every tensor), copies each piece in on
+ * an internal host-to-device stream, computes it on `stream` as a problem of
+ * its own (B = 1; the result equals favor_attention(_f32) on those heads bit
+ * for bit) and copies it out on an internal device-to-host stream, so that both
+ * copy directions and the compute overlap.  It synchronises `stream` before
+ * returning.  Device buffers (two pieces' tensors, W, one piece's scratch) are
+ * allocated and freed stream-ordered on `stream` inside the call; the two copy
+ * streams are created on first use per device and kept for the process.
  */
 FAVOR_API int favor_attention_host(int dtype, const void* Q, const void* K, const void* V, const float* W,
                          void* out, int B, int H, int Hkv, int L, int d, int m,

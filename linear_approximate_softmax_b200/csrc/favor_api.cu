@@ -5,7 +5,9 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "favor_internal.h"
 
@@ -171,6 +173,24 @@ void keep_pool_mapped() {
   done[dev] = true;
 }
 
+// The host-buffer call's copy streams on each device (host to device, device to host),
+// created on first use and kept for the process, so that the two copy directions run on
+// their own copy engines beside the compute on the caller's stream.
+int copy_streams(cudaStream_t* in, cudaStream_t* out) {
+  static std::mutex mu;
+  static cudaStream_t streams[64][2] = {};
+  int dev = 0;
+  FAVOR_CUDA_TRY(cudaGetDevice(&dev), "favor_attention_host device");
+  if (dev < 0 || dev >= 64) return set_error(FAVOR_ERR_UNSUPPORTED, "favor_attention_host: device index above 63");
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < 2; ++i)
+    if (!streams[dev][i])
+      FAVOR_CUDA_TRY(cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking), "favor_attention_host streams");
+  *in = streams[dev][0];
+  *out = streams[dev][1];
+  return FAVOR_OK;
+}
+
 int attention_impl(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,
                    int H, int Hkv, int L, int d, int m, cudaStream_t st) {
   FAVOR_TRY(check_dtype(dtype));
@@ -222,32 +242,111 @@ int favor_attention_host(int dtype, const void* Q, const void* K, const void* V,
   if (!Q || !K || !V || !W || !out) return set_error(FAVOR_ERR_INVALID, "favor_attention_host: null pointer argument");
   FAVOR_TRY(check_shape(B, H, Hkv, L, d, m));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  FAVOR_TRY(copy_streams(&s_in, &s_out));
+  // Pieces of consecutive kv heads (each with its G query heads): kv head t = b * Hkv + j owns
+  // query heads t * G .. t * G + G - 1 in the [B, H] order, so a piece is one contiguous range of
+  // Q, K, V and out and is computed as a problem of its own (B = 1).  Piece i goes in on s_in,
+  // is computed on the caller's stream and goes out on s_out, double-buffered on the device, so
+  // the copies of neighbouring pieces overlap each other (both directions) and the compute.
+  const int G = H / Hkv, KH = B * Hkv;
+  const int NP = KH < 8 ? KH : 8;
+  const int nmax = (KH + NP - 1) / NP;
   const size_t es = dtype == FAVOR_F32 ? 4 : 2;
-  const size_t nq = static_cast<size_t>(B) * H * L * d, nk = static_cast<size_t>(B) * Hkv * L * d;
-  const size_t bq = round_up(nq * es, 256), bk = round_up(nk * es, 256), bw = round_up(sizeof(float) * m * d, 256);
-  void* buf = nullptr;
+  const size_t row = static_cast<size_t>(L) * d * es;  // one head of one tensor
+  const size_t bkv = round_up(nmax * row, 256), bq = round_up(nmax * G * row, 256);
+  const size_t bw = round_up(sizeof(float) * m * d, 256);
+  auto piece = [&](int i, int* t0, int* n) {
+    *t0 = static_cast<int>(static_cast<long>(KH) * i / NP);
+    *n = static_cast<int>(static_cast<long>(KH) * (i + 1) / NP) - *t0;
+  };
+  size_t part_max = 0, st_max = 0;  // one scratch for every piece's partials and state
+  for (int i = 0; i < NP; ++i) {
+    int t0, n;
+    piece(i, &t0, &n);
+    Plan pp;
+    FAVOR_TRY(make_plan(1, n * G, n, L, d, m, &pp));
+    part_max = pp.part_bytes > part_max ? pp.part_bytes : part_max;
+    st_max = pp.st_bytes > st_max ? pp.st_bytes : st_max;
+  }
+  const size_t st_off = round_up(part_max, 256);
+  const size_t scratch = st_off + round_up(st_max, 256);
+  const size_t slot = 2 * bkv + 2 * bq;  // K, V, Q, out of one piece
   keep_pool_mapped();
-  FAVOR_CUDA_TRY(cudaMallocAsync(&buf, 2 * bq + 2 * bk + bw, st), "favor_attention_host device allocation");
-  char* dQ = static_cast<char*>(buf);
-  char* dK = dQ + bq;
-  char* dV = dK + bk;
-  char* dW = dV + bk;
-  char* dO = dW + bw;
+  void* buf = nullptr;
+  FAVOR_CUDA_TRY(cudaMallocAsync(&buf, bw + scratch + 2 * slot, st), "favor_attention_host device allocation");
+  char* dW = static_cast<char*>(buf);
+  char* dS = dW + bw;
+  std::vector<cudaEvent_t> ev(3 * NP + 1, nullptr);  // ready, then per piece: in, computed, out
+  cudaError_t e = cudaSuccess;
+  for (auto& x : ev)
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+  auto ev_in = [&](int i) { return ev[1 + 3 * i]; };
+  auto ev_comp = [&](int i) { return ev[2 + 3 * i]; };
+  auto ev_out = [&](int i) { return ev[3 + 3 * i]; };
   int rc = FAVOR_OK;
-  cudaError_t e = cudaMemcpyAsync(dQ, Q, nq * es, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dK, K, nk * es, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dV, V, nk * es, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dW, W, sizeof(float) * m * d, cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) rc = set_errorf(FAVOR_ERR_CUDA, "favor_attention_host copy in: %s", cudaGetErrorString(e));
-  if (rc == FAVOR_OK)
-    rc = attention_impl(dtype, dQ, dK, dV, reinterpret_cast<const float*>(dW), dO, B, H, Hkv, L, d, m, st);
-  if (rc == FAVOR_OK) {
-    e = cudaMemcpyAsync(out, dO, nq * es, cudaMemcpyDeviceToHost, st);
-    if (e != cudaSuccess) rc = set_errorf(FAVOR_ERR_CUDA, "favor_attention_host copy out: %s", cudaGetErrorString(e));
+  if (e == cudaSuccess) e = cudaEventRecord(ev[0], st);  // the allocation (and all earlier work on st)
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev[0], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev[0], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dW, W, sizeof(float) * m * d, cudaMemcpyHostToDevice, s_in);
+  if (e != cudaSuccess) rc = set_errorf(FAVOR_ERR_CUDA, "favor_attention_host set-up: %s", cudaGetErrorString(e));
+  for (int i = 0; i < NP && rc == FAVOR_OK; ++i) {
+    int t0, n;
+    piece(i, &t0, &n);
+    char* sK = dS + scratch + (i & 1) * slot;
+    char* sV = sK + bkv;
+    char* sQ = sV + bkv;
+    char* sO = sQ + bq;
+    const size_t nkv = n * row, nq = static_cast<size_t>(n) * G * row;
+    if (i >= 2) e = cudaStreamWaitEvent(s_in, ev_comp(i - 2), 0);  // piece i - 2 has read this slot
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sK, static_cast<const char*>(K) + t0 * row, nkv, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sV, static_cast<const char*>(V) + t0 * row, nkv, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(sQ, static_cast<const char*>(Q) + static_cast<size_t>(t0) * G * row, nq, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in(i), s_in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev_in(i), 0);
+    if (e == cudaSuccess && i >= 2) e = cudaStreamWaitEvent(st, ev_out(i - 2), 0);  // this slot's output has left
+    if (e != cudaSuccess) {
+      rc = set_errorf(FAVOR_ERR_CUDA, "favor_attention_host copy in: %s", cudaGetErrorString(e));
+      break;
+    }
+    Plan pp;
+    rc = make_plan(1, n * G, n, L, d, m, &pp);
+    const float* w = reinterpret_cast<const float*>(dW);
+    if (rc == FAVOR_OK) rc = run_key_pass(dtype, sK, sV, w, dS, pp, st);
+    if (rc == FAVOR_OK) rc = run_reduce(dS, dS + st_off, pp, st);
+    if (rc == FAVOR_OK) rc = run_query_pass(dtype, sQ, w, dS + st_off, sO, pp, st);
+    if (rc != FAVOR_OK) break;
+    e = cudaEventRecord(ev_comp(i), st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_comp(i), 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<char*>(out) + static_cast<size_t>(t0) * G * row, sO, nq, cudaMemcpyDeviceToHost, s_out);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_out(i), s_out);
+    if (e != cudaSuccess) {
+      rc = set_errorf(FAVOR_ERR_CUDA, "favor_attention_host copy out: %s", cudaGetErrorString(e));
+      break;
+    }
+  }
+  // join both copy streams into the caller's stream (also after an error), then release
+  cudaEvent_t jin = nullptr, jout = nullptr;
+  cudaError_t je = cudaEventCreateWithFlags(&jin, cudaEventDisableTiming);
+  if (je == cudaSuccess) je = cudaEventCreateWithFlags(&jout, cudaEventDisableTiming);
+  if (je == cudaSuccess) je = cudaEventRecord(jin, s_in);
+  if (je == cudaSuccess) je = cudaEventRecord(jout, s_out);
+  if (je == cudaSuccess) je = cudaStreamWaitEvent(st, jin, 0);
+  if (je == cudaSuccess) je = cudaStreamWaitEvent(st, jout, 0);
+  if (je != cudaSuccess) {  // cannot order the release after the copies: wait for them here
+    cudaStreamSynchronize(s_in);
+    cudaStreamSynchronize(s_out);
   }
   cudaError_t fe = cudaFreeAsync(buf, st);
   cudaError_t se = cudaStreamSynchronize(st);
+  for (auto& x : ev)
+    if (x) cudaEventDestroy(x);
+  if (jin) cudaEventDestroy(jin);
+  if (jout) cudaEventDestroy(jout);
   if (rc != FAVOR_OK) return rc;
+  if (je != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "favor_attention_host join: %s", cudaGetErrorString(je));
   if (fe != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "favor_attention_host release: %s", cudaGetErrorString(fe));
   if (se != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "favor_attention_host: %s", cudaGetErrorString(se));
   return FAVOR_OK;

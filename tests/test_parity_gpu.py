@@ -199,6 +199,26 @@ def test_stage_calls_equal_fused_call_and_state_matches_oracle(dtype):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_host_call_pieces_equal_device_calls(dtype):
+    # ten kv heads: the host call splits them into eight pieces of consecutive kv heads (sizes 1
+    # and 2, one piece across a batch boundary) and runs each as a problem of its own, so each
+    # piece must equal the device call on the same heads bit for bit
+    B, H, Hkv, L, d, m = 5, 4, 2, 200, 64, 64
+    G, KH, NP = H // Hkv, B * Hkv, 8
+    Q, K, V = wl.random_inputs(B, H, Hkv, L, d, dtype, seed=9)
+    W = fv.favor_make_features(2, m, d)
+    host = fv.favor_attention_host(Q.pin_memory(), K.pin_memory(), V.pin_memory(), W)
+    Qf, Kf, Vf, Of = (x.reshape(-1, L, d) for x in (Q, K, V, host))
+    spans = []
+    for i in range(NP):
+        t0, t1 = KH * i // NP, KH * (i + 1) // NP
+        spans.append((t0, t1))
+        dev = gpu_attention(Qf[t0 * G:t1 * G][None], Kf[t0:t1][None], Vf[t0:t1][None], W)
+        assert torch.equal(Of[t0 * G:t1 * G], dev[0].cpu()), (i, t0, t1)
+    assert any(t0 // Hkv != (t1 - 1) // Hkv for t0, t1 in spans)  # a piece spans two batches
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_host_call_equals_device_call(dtype):
     Q, K, V = wl.random_inputs(1, 2, 1, 777, 128, dtype, seed=5)
     W = fv.favor_make_features(1, 128, 128)
