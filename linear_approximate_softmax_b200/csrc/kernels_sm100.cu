@@ -746,6 +746,32 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
 // ============================================================================
 // Query pass
 // ============================================================================
+// Where a query tile lies: query head bh (= b * H + h), 128-row tile qt within it, gq = bh % G and
+// its state image, kv head bh / G (H = Hkv * G) counted from the CTA's first kv head.  Each role
+// walks its tiles in fixed steps, so the cursor advances by additions: a division by a runtime
+// value costs tens of dependent instructions, which the issuing and epilogue threads would pay
+// on every tile or block.
+struct TileCursor {
+  int bh, qt, gq, img;
+  __device__ __forceinline__ void init(int T, int ntq, int G, int kvh0) {
+    bh = T / ntq;
+    qt = T - bh * ntq;
+    gq = bh % G;
+    img = bh / G - kvh0;
+  }
+  __device__ __forceinline__ void step(int by, int ntq, int G) {
+    qt += by;
+    while (qt >= ntq) {
+      qt -= ntq;
+      ++bh;
+      if (++gq == G) {
+        gq = 0;
+        ++img;
+      }
+    }
+  }
+};
+
 template <int D>
 struct QueryCfg {
   // warp 0 TMA producer, warps 1-2 MMA issuers (one per warpgroup), warp 3 idle,
@@ -814,15 +840,10 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
   uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
   auto bar = [&](int i) { return sbase + C::S_BAR + 8u * i; };
-  // kv head of a tile; non-decreasing along the tile order, so the CTA's tiles visit each
-  // kv head once: image index of local tile t = img(t), 0 .. nimg - 1
-  auto kvh_of = [&](int T) {
-    const int bh = T / ntq;
-    return (bh / H) * Hkv + (bh % H) / G;
-  };
-  const int kvh0 = kvh_of(T0);
-  auto img = [&](int t) { return kvh_of(T0 + t) - kvh0; };
-  const int nimg = n > 0 ? img(n - 1) + 1 : 0;
+  // kv head of a tile (b * Hkv + h / G = (b * H + h) / G); non-decreasing along the tile order,
+  // so the CTA's tiles visit each kv head once: image index 0 .. nimg - 1
+  const int kvh0 = T0 / ntq / G;
+  const int nimg = n > 0 ? (T0 + n - 1) / ntq / G - kvh0 + 1 : 0;
 
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -900,18 +921,20 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     // ---------------- producer: Q tiles (stage = tile parity) and state images ----------------
     if (lane == 0) {
       int loaded = n > 0 ? 0 : -1, issued = 0;  // tiles 0 and 1 and image 0 were issued during the set-up
-      for (int it = 0; it < n; ++it) {
-        const int T = T0 + it, s = it & 1;
+      TileCursor pc;
+      pc.init(T0, ntq, G, kvh0);
+      for (int it = 0; it < n; ++it, pc.step(1, ntq, G)) {
+        const int s = it & 1;
         if (it >= 2) {
           if (!mbar_wait<true>(bar(C::B_QE + s), ((it >> 1) - 1) & 1, abort_flag, err)) break;
           mbar_arrive_expect_tx(bar(C::B_QF + s), C::QTILE);
-          const int bh = T / ntq, qt = T % ntq;
 #pragma unroll
           for (int r = 0; r < D / 64; ++r)
-            tma_load_3d(sbase + C::S_Q + s * C::QTILE + r * (128 * 128), &tmQ, bar(C::B_QF + s), 64 * r, qt * 128, bh);
+            tma_load_3d(sbase + C::S_Q + s * C::QTILE + r * (128 * 128), &tmQ, bar(C::B_QF + s), 64 * r, pc.qt * 128,
+                        pc.bh);
         }
         issued = it + 1;
-        const int k = img(it);
+        const int k = pc.img;
         if (k > loaded) {  // a new kv head: load its image once both issuers have released the previous one
           if (k >= 1 && !mbar_wait(bar(C::B_SE), (k - 1) & 1, abort_flag, err)) break;
           mbar_arrive_expect_tx(bar(C::B_SF), op_bytes);
@@ -948,8 +971,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       // U = (2^-k Q) W'^T in fp16 for my block b, always FB columns wide: W' rows past m are
       // zero, so every U column the epilogue reads is written (its e = -inf masks it)
       const uint32_t id1 = idesc_f16(128, FB, false, false);
-      auto mma1 = [&](int b) {
-        const int j = b % nb;
+      auto mma1 = [&](int j) {
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t qo = (ks >> 2) * (128 * 128) + 32 * (ks & 3);
@@ -962,27 +984,27 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       };
       // before the first projection of my tile tcn: release the images that precede its image
       // and that I never used, then wait for its Q to be converted
-      auto enter_tile = [&](int tcn) {
-        const int kn = img(w + 2 * tcn);
+      auto enter_tile = [&](int tcn, int kn) {
         while (rel < kn)
           if (!release_unused()) return false;
         return mbar_wait(bar(C::B_CVT + w), tcn & 1, abort_flag, err);
       };
+      TileCursor cur;  // my tile t = w + 2 * tc
       if (nblk > 0) {
-        ok = enter_tile(0);
+        cur.init(T0 + w, ntq, G, kvh0);
+        ok = enter_tile(0, cur.img);
         if (ok) {
           tc_fence_after();
           mma1(0);
         }
       }
-      for (int b = 0; b < nblk && ok; ++b) {
-        const int tc = b / nb, j = b % nb, t = w + 2 * tc;
-        const int k = img(t);
+      for (int b = 0, tc = 0, j = 0; b < nblk && ok; ++b) {
+        const int t = w + 2 * tc, k = cur.img;
         const bool more = b + 1 < nblk, boundary = (j == nb - 1);
         if (more && !boundary) {  // next block of the same tile
           if (!mbar_wait(bar(C::B_UE + w), b & 1, abort_flag, err)) break;
           tc_fence_after();
-          mma1(b + 1);
+          mma1(j + 1);
         }
         if (!mbar_wait(bar(C::B_PHI + w), b & 1, abort_flag, err)) break;
         if (j == 0) {
@@ -999,17 +1021,24 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         mma_commit(bar(C::B_M2 + w));
         if (boundary) {
           mma_commit(bar(C::B_OF + w));
-          const int knext = t + 2 < n ? img(t + 2) : nimg;
+          TileCursor nx = cur;  // my next tile, t + 2
+          nx.step(2, ntq, G);
+          const int knext = t + 2 < n ? nx.img : nimg;
           if (knext > k && k < nimg - 1) {  // done with image k: released when these MMAs complete
             mma_commit(bar(C::B_SE));
             rel = k + 1;
           }
           if (more) {  // first block of my next tile: U read and that tile's Q converted
             if (!mbar_wait(bar(C::B_UE + w), b & 1, abort_flag, err)) break;
-            if (!enter_tile(tc + 1)) break;
+            if (!enter_tile(tc + 1, nx.img)) break;
             tc_fence_after();
-            mma1(b + 1);
+            mma1(0);
           }
+          cur = nx;
+          ++tc;
+          j = 0;
+        } else {
+          ++j;
         }
       }
       while (ok && rel < nimg - 1) ok = release_unused();
@@ -1075,9 +1104,11 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     };
     float up_next = ewg < n ? prepare(0) : 1.f;
     int cntb = 0, tc = 0;
-    for (int t = ewg; t < n; t += 2, ++tc) {
+    TileCursor ec;  // my tile t
+    if (ewg < n) ec.init(T0 + ewg, ntq, G, kvh0);
+    for (int t = ewg; t < n; t += 2, ++tc, ec.step(2, ntq, G)) {
       const float up = up_next;
-      mbar_wait(bar(C::B_SF), img(t) & 1, abort_flag, err);  // this tile's image (exponents) is in
+      mbar_wait(bar(C::B_SF), ec.img & 1, abort_flag, err);  // this tile's image (exponents) is in
       float c = 0.f, den = 0.f;
       for (int j = 0; j < nb; ++j, ++cntb) {
         mbar_wait(bar(C::B_UF + ewg), cntb & 1, abort_flag, err);
@@ -1156,7 +1187,6 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       } else {  // the slot is free once the same quarter of tile t - 1 has been stored
         if (t >= 1) mbar_wait(bar(C::B_STG + eq), (t - 1) & 1, abort_flag, err);
       }
-      const int T = T0 + t, bh = T / ntq, qt = T % ntq;
 #pragma unroll
       for (int rg = 0; rg < D / 64; ++rg) {
         if (rg > 0) {  // the previous region's store has read the slot
@@ -1187,7 +1217,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tmO, smem_u32(slot), 64 * rg, qt * 128 + 32 * eq, bh);
+          tma_store_3d(&tmO, smem_u32(slot), 64 * rg, ec.qt * 128 + 32 * eq, ec.bh);
           bulk_commit();
         }
       }
