@@ -234,21 +234,27 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+  // amax = mant * 2^(ex + 15), mant in [0.5, 1), so amax * 2^-ex lies in [2^14, 2^15)
   int ex = 0;
-  if (amax > 0.f) {
-    frexpf(amax, &ex);  // amax = mant * 2^ex, mant in [0.5, 1)
-    ex -= 15;           // amax * 2^-ex in [2^14, 2^15)
+  if (amax >= 1.17549435e-38f) {
+    ex = ((__float_as_int(amax) >> 23) & 0xFF) - 126 - 15;
+  } else if (amax > 0.f) {  // subnormal
+    frexpf(amax, &ex);
+    ex -= 15;
   }
+  // 2^-ex as two normal factors (|ex| <= 164), an exact scaling wherever the result is normal
+  const int ea = -ex / 2, eb = -ex - ea;
+  const float sa = __int_as_float((127 + ea) << 23), sb = __int_as_float((127 + eb) << 23);
 #pragma unroll
   for (int k = 0; k < NC; ++k) {
     const int n = g + 8 * k;
-    if (n < D) stage[n][fl] = __float2half_rn(ldexpf(val[k], -ex));
+    if (n < D) stage[n][fl] = __float2half_rn(val[k] * sa * sb);
   }
   unsigned char* img = op + static_cast<size_t>(head) * op_bytes;
   // tail: the exponent of each feature, then its normaliser entry with the same scaling
   float* tail = reinterpret_cast<float*>(img + static_cast<size_t>(D) * 128 * op_atoms);
   if (g == 0) tail[f] = live && cf > -INFINITY ? static_cast<float>(ex) + (cf - cs) : -INFINITY;
-  if ((D & 7) == g) tail[op_tail + f] = live ? ldexpf(den, -ex) : 0.f;
+  if ((D & 7) == g) tail[op_tail + f] = live ? den * sa * sb : 0.f;
   __syncthreads();
   // the image holds 64 features per 128-byte row (dimension n), 16-byte chunk c at c ^ (n % 8):
   // this CTA's 32 features are four chunks of each row of its 64-feature atom
