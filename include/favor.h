@@ -25,6 +25,13 @@
  *  - GPU entry points are asynchronous on `stream` (0 = legacy default
  *    stream) and never synchronise it; CUDA launch errors are reported as
  *    FAVOR_ERR_CUDA.
+ *  - The tensor-core kernels and the state reduction are launched with
+ *    programmatic dependent launch, so each may start while the kernel before
+ *    it on `stream` finishes; each waits (griddepcontrol.wait) before it reads
+ *    or overwrites memory that an earlier kernel uses.  Work the caller adds to
+ *    `stream` afterwards is ordered after them as usual; a kernel the caller
+ *    itself launches with programmatic stream serialisation must wait the same
+ *    way before it reads their outputs.
  *  - Supported shapes: d in {64, 128}; m a multiple of 16 with 16 <= m <= 512;
  *    B, H, Hkv, L >= 1; H % Hkv == 0.  Anything else is FAVOR_ERR_UNSUPPORTED.
  */
