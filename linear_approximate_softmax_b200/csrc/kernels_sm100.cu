@@ -28,6 +28,12 @@
 //   out = O / (phi' . s) -> bf16 -> TMA store.
 // The state image holds each feature row scaled by its own power of two, so that fp16
 // keeps 11 bits for every row; adding e_f to the exponent restores the product.
+// Each role walks its tiles with a cursor that advances by additions (no division by a
+// runtime value on the per-tile or per-block path).
+//
+// Both kernels are launched with programmatic dependent launch (launch.cuh): they let the
+// next kernel on the stream be scheduled at once and wait (griddepcontrol.wait) only before
+// storing the partial state (key pass) or loading the first state image (query pass).
 //
 // Every mbarrier wait is bounded (2 s); a CTA that gives up raises the device
 // error word, stops issuing work, drains its own copies and frees its TMEM.
