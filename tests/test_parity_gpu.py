@@ -167,6 +167,31 @@ def test_deterministic_bitwise():
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("H,Hkv,d", [(8, 8, 64), (8, 1, 128)])
+def test_back_to_back_calls_reusing_scratch(H, Hkv, d):
+    # Three stage sequences issued back to back on one stream with no synchronisation, all
+    # sharing one partial-state and one state buffer.  The kernels are launched so that each
+    # may start while the one before it finishes; each must still wait before it overwrites a
+    # buffer an earlier kernel reads (the next key pass's partials, the next reduction's state),
+    # so every output equals the same call made alone, bit for bit.
+    B, L, m = 2, 8192, 256
+    W = fv.favor_make_features(3, m, d).cuda()
+    sets = [[t.cuda() for t in wl.random_inputs(B, H, Hkv, L, d, torch.bfloat16, seed=20 + i)] for i in range(3)]
+    part = torch.empty(fv.favor_partials_bytes(B, Hkv, L, d, m), dtype=torch.uint8, device="cuda")
+    state = torch.empty(fv.favor_state_bytes(B, Hkv, d, m), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty_like(q) for q, _, _ in sets]
+    for (Qd, Kd, Vd), out in zip(sets, outs):
+        fv.favor_key_pass(Kd, Vd, W, part)
+        fv.favor_state_reduce(part, state, B, Hkv, L, d, m)
+        fv.favor_query_pass(Qd, W, state, Hkv, out)
+    fv.favor_device_check()
+    for (Qd, Kd, Vd), out in zip(sets, outs):
+        alone = fv.favor_attention(Qd, Kd, Vd, W)
+        fv.favor_device_check()
+        assert torch.equal(out, alone)
+    assert not torch.equal(outs[0], outs[1])
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_stage_calls_equal_fused_call_and_state_matches_oracle(dtype):
     B, H, Hkv, L, d, m = 2, 4, 2, 1500, 64, 192
