@@ -33,7 +33,8 @@
  *    itself launches with programmatic stream serialisation must wait the same
  *    way before it reads their outputs.
  *  - Supported shapes: d in {64, 128}; m a multiple of 16 with 16 <= m <= 512;
- *    B, H, Hkv, L >= 1; H % Hkv == 0.  Anything else is FAVOR_ERR_UNSUPPORTED.
+ *    B, H, Hkv, L >= 1; H % Hkv == 0; B * H <= 65535.  Anything else is
+ *    FAVOR_ERR_UNSUPPORTED.
  */
 #ifndef FAVOR_B200_H
 #define FAVOR_B200_H

@@ -25,6 +25,9 @@ int check_shape(int B, int H, int Hkv, int L, int d, int m) {
   if (d != 64 && d != 128) return set_errorf(FAVOR_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
   if (m < 16 || m > 512 || m % 16 != 0)
     return set_errorf(FAVOR_ERR_UNSUPPORTED, "m must be a multiple of 16 in [16, 512] (got %d)", m);
+  // the kernels index (batch, head) pairs with a grid dimension of at most 65535
+  if (static_cast<long>(B) * H > 65535)
+    return set_errorf(FAVOR_ERR_UNSUPPORTED, "B * H must be at most 65535 (got %ld)", static_cast<long>(B) * H);
   const double elems = static_cast<double>(B) * H * L * d;
   if (elems > 4.0e12) return set_error(FAVOR_ERR_UNSUPPORTED, "tensor too large");
   return FAVOR_OK;

@@ -354,7 +354,7 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   auto kern = key_pass_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "key pass attribute: %s", cudaGetErrorString(e));
-  dim3 grid(p.P, p.B * p.Hkv, p.nsb);
+  dim3 grid(p.P, p.B * p.Hkv, (p.m + kFB - 1) / kFB);
   char* base = static_cast<char*>(partials);
   kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(K), static_cast<const T*>(V), W,
                                      reinterpret_cast<float*>(base + p.part_S_off),

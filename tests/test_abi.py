@@ -73,6 +73,7 @@ def attn(ptrs, B=1, H=1, Hkv=1, L=16, d=64, m=64):
     (dict(H=3, Hkv=2), fv.FAVOR_ERR_UNSUPPORTED),
     (dict(L=0), fv.FAVOR_ERR_UNSUPPORTED),
     (dict(B=0), fv.FAVOR_ERR_UNSUPPORTED),
+    (dict(B=4096, H=16, Hkv=16), fv.FAVOR_ERR_UNSUPPORTED),  # B * H above the grid limit
 ])
 def test_attention_rejects_unsupported_shapes(shape, code):
     assert attn([FAKE] * 5, **shape) == code
