@@ -98,3 +98,9 @@ def test_stage_calls_reject_bad_dtype_and_pointers():
 def test_valid_call_without_a_device_reports_cuda_error():
     assert attn([FAKE] * 5) == fv.FAVOR_ERR_CUDA
     assert fv.favor_partials_bytes(1, 1, 16, 64, 64) == 0
+    # the host-buffer call fails cleanly before it copies anything
+    q = np.zeros(16 * 64, np.uint16)
+    w = np.zeros(64 * 64, np.float32)
+    ptr = lambda x: ctypes.c_void_p(x.ctypes.data)  # noqa: E731
+    rc = fv.lib.favor_attention_host(fv.FAVOR_BF16, ptr(q), ptr(q), ptr(q), ptr(w), ptr(q.copy()), 1, 1, 1, 16, 64, 64, None)
+    assert rc == fv.FAVOR_ERR_CUDA and fv.lib.favor_last_error()
