@@ -238,6 +238,9 @@ def main():
         return
 
     import linear_approximate_softmax_b200 as fv
+    # every kernel on this stream is the library's own, none lets its dependents start early:
+    # the first kernel of each call may overlap the end of the previous call (favor.h)
+    fv.favor_set_launch_overlap(True)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = wl.WORKLOADS[args.workload]
@@ -333,7 +336,7 @@ def main():
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "L": w.L, "d": w.d, "m": w.m,
-                   "parallelism": f"replicas x{world}",
+                   "parallelism": f"replicas x{world}", "launch_overlap": True,
                    "l2": f"inputs larger than L2 ({(Qh.numel() + Kh.numel() + Vh.numel()) * elt / 1e6:.0f} MB of Q,K,V per step)"},
         "roofline": {"kernel": names[dom], "bound": "alu", "achieved": achieved,
                      "peak": rt["mufu_peak_gexps"], "unit": "Gexp/s", "frac": achieved / rt["mufu_peak_gexps"],

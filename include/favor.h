@@ -25,13 +25,15 @@
  *  - GPU entry points are asynchronous on `stream` (0 = legacy default
  *    stream) and never synchronise it; CUDA launch errors are reported as
  *    FAVOR_ERR_CUDA.
- *  - The tensor-core kernels and the state reduction are launched with
- *    programmatic dependent launch, so each may start while the kernel before
- *    it on `stream` finishes; each waits (griddepcontrol.wait) before it reads
- *    or overwrites memory that an earlier kernel uses.  Work the caller adds to
- *    `stream` afterwards is ordered after them as usual; a kernel the caller
- *    itself launches with programmatic stream serialisation must wait the same
- *    way before it reads their outputs.
+ *  - Within one call, the state reduction and the tensor-core query pass are
+ *    launched with programmatic dependent launch: each may start while the
+ *    call's kernel before it finishes, and waits (griddepcontrol.wait) before
+ *    it reads or overwrites memory that kernel uses.  The first kernel of a
+ *    call is an ordinary launch (it starts once all earlier work on `stream`
+ *    has completed) unless favor_set_launch_overlap(1) was called.  Work the
+ *    caller adds to `stream` afterwards is ordered after the call as usual; a
+ *    kernel the caller launches with programmatic stream serialisation must
+ *    wait the same way before it reads the call's outputs.
  *  - Supported shapes: d in {64, 128}; m a multiple of 16 with 16 <= m <= 512;
  *    B, H, Hkv, L >= 1; H % Hkv == 0; B * H <= 65535.  Anything else is
  *    FAVOR_ERR_UNSUPPORTED.
@@ -64,6 +66,22 @@ typedef struct CUstream_st* favor_stream_t; /* the same type as cudaStream_t */
 /* Element type of Q, K, V and out. */
 #define FAVOR_BF16 0
 #define FAVOR_F32 1
+
+/*
+ * favor_set_launch_overlap — how the first kernel of every later call starts
+ * (process-wide; returns the previous setting, 0 or 1).
+ *
+ * 0 (the default): an ordinary launch, after all earlier work on the stream.
+ * 1: a programmatic dependent launch, like the later kernels of a call: it may
+ * start as soon as the kernel before it on the stream lets its dependents start
+ * (griddepcontrol.launch_dependents) or exits, and it reads its inputs (Q, K, V,
+ * W, or a stage call's partial state or state) at once.  Enable it only if no
+ * kernel placed on a stream before a library call lets its dependents start
+ * before its writes are complete; kernels that do not use programmatic
+ * dependent launch never do.  A call's set-up then overlaps the end of the
+ * kernel before it (for back-to-back calls, the previous query pass).
+ */
+FAVOR_API int favor_set_launch_overlap(int enable);
 
 /* Message for the last non-zero return on the calling thread ("" if none). */
 FAVOR_API const char* favor_last_error(void);

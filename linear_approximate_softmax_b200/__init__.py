@@ -29,6 +29,7 @@ EXPORTS = [
     "favor_last_error", "favor_version", "favor_make_features", "favor_attention",
     "favor_attention_f32", "favor_attention_host", "favor_partials_bytes", "favor_state_bytes",
     "favor_key_pass", "favor_state_reduce", "favor_query_pass", "favor_attention_noalloc", "favor_device_check",
+    "favor_set_launch_overlap",
 ]
 
 if not os.path.exists(LIB_PATH):
@@ -62,6 +63,14 @@ lib.favor_device_check.argtypes = [_p]
 lib.favor_device_check.restype = _i
 lib.favor_attention_noalloc.argtypes = [_i] + _ATT
 lib.favor_attention_noalloc.restype = _i
+lib.favor_set_launch_overlap.argtypes = [_i]
+lib.favor_set_launch_overlap.restype = _i
+
+
+def favor_set_launch_overlap(enable):
+    """Whether the first kernel of each later call may start while the kernel before it on the
+    stream finishes (see favor.h); returns the previous setting."""
+    return bool(lib.favor_set_launch_overlap(1 if enable else 0))
 
 
 class FavorError(RuntimeError):

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -144,20 +145,26 @@ void plan_limit_chunks(Plan* p, int max_P) {
 }
 
 int run_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials, const Plan& p,
-                 cudaStream_t st) {
-  if (dtype == FAVOR_BF16 && sm100_key_supported(p)) return sm100_key_pass(K, V, W, partials, p, st);
-  return simt_key_pass(dtype, K, V, W, partials, p, st);
+                 cudaStream_t st, bool overlap) {
+  if (dtype == FAVOR_BF16 && sm100_key_supported(p)) return sm100_key_pass(K, V, W, partials, p, st, overlap);
+  return simt_key_pass(dtype, K, V, W, partials, p, st);  // an ordinary launch
 }
 
-int run_reduce(const void* partials, void* state, const Plan& p, cudaStream_t st) {
-  return simt_state_reduce(partials, state, p, st);
+int run_reduce(const void* partials, void* state, const Plan& p, cudaStream_t st, bool overlap) {
+  return simt_state_reduce(partials, state, p, st, overlap);
 }
 
 int run_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out, const Plan& p,
-                   cudaStream_t st) {
-  if (dtype == FAVOR_BF16 && sm100_query_supported(p)) return sm100_query_pass(Q, W, state, out, p, st);
-  return simt_query_pass(dtype, Q, W, state, out, p, st);
+                   cudaStream_t st, bool overlap) {
+  if (dtype == FAVOR_BF16 && sm100_query_supported(p)) return sm100_query_pass(Q, W, state, out, p, st, overlap);
+  return simt_query_pass(dtype, Q, W, state, out, p, st);  // an ordinary launch
 }
+
+namespace {
+std::atomic<int> g_launch_overlap{0};
+}  // namespace
+
+bool launch_overlap_enabled() { return g_launch_overlap.load(std::memory_order_relaxed) != 0; }
 
 namespace {
 
@@ -205,9 +212,9 @@ int attention_impl(int dtype, const void* Q, const void* K, const void* V, const
   const size_t st_off = round_up(p.part_bytes, 256);
   FAVOR_CUDA_TRY(cudaMallocAsync(&ws, st_off + p.st_bytes, st), "favor_attention scratch allocation");
   char* base = static_cast<char*>(ws);
-  int rc = run_key_pass(dtype, K, V, W, base, p, st);
-  if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, p, st);
-  if (rc == FAVOR_OK) rc = run_query_pass(dtype, Q, W, base + st_off, out, p, st);
+  int rc = run_key_pass(dtype, K, V, W, base, p, st, launch_overlap_enabled());
+  if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, p, st, true);
+  if (rc == FAVOR_OK) rc = run_query_pass(dtype, Q, W, base + st_off, out, p, st, true);
   cudaError_t fe = cudaFreeAsync(ws, st);
   if (rc != FAVOR_OK) return rc;
   FAVOR_CUDA_TRY(fe, "favor_attention scratch release");
@@ -224,6 +231,10 @@ extern "C" {
 const char* favor_last_error(void) { return g_last_error.c_str(); }
 
 int favor_version(void) { return 100; }
+
+int favor_set_launch_overlap(int enable) {
+  return g_launch_overlap.exchange(enable ? 1 : 0, std::memory_order_relaxed);
+}
 
 int favor_make_features(uint64_t seed, int m, int d, int orthogonal, float* W_out) {
   return make_features(seed, m, d, orthogonal, W_out);
@@ -316,9 +327,10 @@ int favor_attention_host(int dtype, const void* Q, const void* K, const void* V,
     Plan pp;
     rc = make_plan(1, n * G, n, L, d, m, &pp);
     const float* w = reinterpret_cast<const float*>(dW);
-    if (rc == FAVOR_OK) rc = run_key_pass(dtype, sK, sV, w, dS, pp, st);
-    if (rc == FAVOR_OK) rc = run_reduce(dS, dS + st_off, pp, st);
-    if (rc == FAVOR_OK) rc = run_query_pass(dtype, sQ, w, dS + st_off, sO, pp, st);
+    // the key pass follows an event wait on the stream: an ordinary launch
+    if (rc == FAVOR_OK) rc = run_key_pass(dtype, sK, sV, w, dS, pp, st, false);
+    if (rc == FAVOR_OK) rc = run_reduce(dS, dS + st_off, pp, st, true);
+    if (rc == FAVOR_OK) rc = run_query_pass(dtype, sQ, w, dS + st_off, sO, pp, st, true);
     if (rc != FAVOR_OK) break;
     e = cudaEventRecord(ev_comp(i), st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_comp(i), 0);
@@ -382,7 +394,7 @@ int favor_key_pass(int dtype, const void* K, const void* V, const float* W, void
   FAVOR_TRY(check_ptrs("favor_key_pass", {K, V, W, partials}));
   Plan p;
   FAVOR_TRY(make_plan(B, Hkv, Hkv, L, d, m, &p));
-  return run_key_pass(dtype, K, V, W, partials, p, reinterpret_cast<cudaStream_t>(stream));
+  return run_key_pass(dtype, K, V, W, partials, p, reinterpret_cast<cudaStream_t>(stream), launch_overlap_enabled());
 }
 
 int favor_state_reduce(const void* partials, void* state, int B, int Hkv, int L, int d, int m,
@@ -390,7 +402,7 @@ int favor_state_reduce(const void* partials, void* state, int B, int Hkv, int L,
   FAVOR_TRY(check_ptrs("favor_state_reduce", {partials, state}));
   Plan p;
   FAVOR_TRY(make_plan(B, Hkv, Hkv, L, d, m, &p));
-  return run_reduce(partials, state, p, reinterpret_cast<cudaStream_t>(stream));
+  return run_reduce(partials, state, p, reinterpret_cast<cudaStream_t>(stream), launch_overlap_enabled());
 }
 
 int favor_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out, int B, int H, int Hkv,
@@ -399,7 +411,8 @@ int favor_query_pass(int dtype, const void* Q, const float* W, const void* state
   FAVOR_TRY(check_ptrs("favor_query_pass", {Q, W, state, out}));
   Plan p;
   FAVOR_TRY(make_plan(B, H, Hkv, L, d, m, &p));
-  return run_query_pass(dtype, Q, W, state, out, p, reinterpret_cast<cudaStream_t>(stream));
+  return run_query_pass(dtype, Q, W, state, out, p, reinterpret_cast<cudaStream_t>(stream),
+                        launch_overlap_enabled());
 }
 
 }  // extern "C"

@@ -52,25 +52,33 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p);
 // recomputes the partials layout (the state layout does not depend on it).
 void plan_limit_chunks(Plan* p, int max_P);
 
-// The three steps of the path, each dispatched to its kernel on `st`.
+// The three steps of the path, each dispatched to its kernel on `st`.  overlap: launch the
+// kernel so that it may start while the kernel before it on `st` finishes (it waits before it
+// touches that kernel's data, but reads its own inputs at once).  Within one call the library
+// sets it for the kernels after the first; for the first kernel of a call it follows
+// launch_overlap_enabled().
 int run_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials, const Plan& p,
-                 cudaStream_t st);
-int run_reduce(const void* partials, void* state, const Plan& p, cudaStream_t st);
+                 cudaStream_t st, bool overlap);
+int run_reduce(const void* partials, void* state, const Plan& p, cudaStream_t st, bool overlap);
 int run_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out, const Plan& p,
-                   cudaStream_t st);
+                   cudaStream_t st, bool overlap);
+// favor_set_launch_overlap's setting (default off).
+bool launch_overlap_enabled();
 
 // ---- CUDA-core kernels (fp32 arithmetic; fp32 or bf16 storage) -------------
 int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void* partials,
                   const Plan& p, void* stream);
-int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream);
+int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream, bool overlap);
 int simt_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out,
                     const Plan& p, void* stream);
 
 // ---- tensor-core kernels (sm_100a, bf16 storage) ------------------------------
 bool sm100_key_supported(const Plan& p);
 bool sm100_query_supported(const Plan& p);
-int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st);
-int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st);
+int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st,
+                   bool overlap);
+int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,
+                     bool overlap);
 // Reads and clears the device error word (bit 0: a bounded wait gave up).
 int sm100_read_and_clear_error(unsigned int* word);
 

@@ -84,8 +84,8 @@ extern "C" int favor_attention_noalloc(int dtype, const void* Q, const void* K, 
   if (rc != FAVOR_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(scratch);
-  rc = run_key_pass(dtype, K, V, W, base, p, st);
-  if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, p, st);
-  if (rc == FAVOR_OK) rc = run_query_pass(dtype, Q, W, base + st_off, out, p, st);
+  rc = run_key_pass(dtype, K, V, W, base, p, st, launch_overlap_enabled());
+  if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, p, st, true);
+  if (rc == FAVOR_OK) rc = run_query_pass(dtype, Q, W, base + st_off, out, p, st, true);
   return rc;
 }

@@ -394,14 +394,14 @@ int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void*
                    : launch_key<__nv_bfloat16, 128>(K, V, W, partials, p, st);
 }
 
-int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream) {
+int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream, bool overlap) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   dim3 grid(p.op_tail / 32, p.B * p.Hkv);
   const char* pb = static_cast<const char*>(partials);
   char* sb = static_cast<char*>(state);
   auto kern = p.d == 64 ? state_reduce_kernel<64> : state_reduce_kernel<128>;
   cudaError_t e = launch_overlapped(
-      kern, grid, dim3(kThreads), 0, st, reinterpret_cast<const float*>(pb + p.part_S_off),
+      kern, grid, dim3(kThreads), 0, st, overlap, reinterpret_cast<const float*>(pb + p.part_S_off),
       reinterpret_cast<const float*>(pb + p.part_c_off), reinterpret_cast<float*>(sb + p.st_S_off),
       reinterpret_cast<float*>(sb + p.st_c_off), reinterpret_cast<unsigned char*>(sb + p.st_op_off), p.P, p.m, p.nsb,
       p.op_atoms, p.op_tail, p.op_bytes);

@@ -1299,7 +1299,8 @@ int check_register_split(const void* kern, int threads) {
 }
 
 template <int D>
-int launch_key(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st) {
+int launch_key(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st,
+               bool overlap) {
   CUtensorMap mk, mv;
   const int heads = p.B * p.Hkv;
   int rc = make_map(&mk, K, D, p.L, heads);
@@ -1323,7 +1324,7 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass attribute: %s", cudaGetErrorString(e));
   char* base = static_cast<char*>(partials);
   dim3 grid((p.m + 127) / 128, p.P, heads);
-  e = launch_overlapped(kern, grid, dim3(threads), smem_bytes, st, mk, mv, W,
+  e = launch_overlapped(kern, grid, dim3(threads), smem_bytes, st, overlap, mk, mv, W,
                         reinterpret_cast<float*>(base + p.part_S_off), reinterpret_cast<float*>(base + p.part_c_off),
                         p.L, p.m, p.P, p.chunk, p.nsb, p.wscale, p.nscale);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass launch: %s", cudaGetErrorString(e));
@@ -1331,7 +1332,8 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
 }
 
 template <int D>
-int launch_query(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st) {
+int launch_query(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,
+                 bool overlap) {
   using C = QueryCfg<D>;
   CUtensorMap mq, mo;
   const int bh = p.B * p.H;
@@ -1346,7 +1348,7 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   const int ntiles = bh * ((p.L + 127) / 128);
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
   const unsigned char* img = static_cast<const unsigned char*>(state) + p.st_op_off;
-  e = launch_overlapped(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, mq, mo, W, img, p.L, p.m, p.H, p.Hkv,
+  e = launch_overlapped(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, overlap, mq, mo, W, img, p.L, p.m, p.H, p.Hkv,
                         ntiles, static_cast<int>(p.op_bytes), p.wscale);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
@@ -1359,12 +1361,16 @@ bool sm100_query_supported(const Plan& p) {
   return (p.d == 64 && p.m <= QueryCfg<64>::MMAX) || (p.d == 128 && p.m <= QueryCfg<128>::MMAX);
 }
 
-int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st) {
-  return p.d == 64 ? launch_key<64>(K, V, W, partials, p, st) : launch_key<128>(K, V, W, partials, p, st);
+int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st,
+                   bool overlap) {
+  return p.d == 64 ? launch_key<64>(K, V, W, partials, p, st, overlap)
+                   : launch_key<128>(K, V, W, partials, p, st, overlap);
 }
 
-int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st) {
-  return p.d == 64 ? launch_query<64>(Q, W, state, out, p, st) : launch_query<128>(Q, W, state, out, p, st);
+int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,
+                     bool overlap) {
+  return p.d == 64 ? launch_query<64>(Q, W, state, out, p, st, overlap)
+                   : launch_query<128>(Q, W, state, out, p, st, overlap);
 }
 
 int sm100_read_and_clear_error(unsigned int* word) {

@@ -80,6 +80,16 @@ def test_attention_rejects_unsupported_shapes(shape, code):
     assert fv.lib.favor_last_error()
 
 
+def test_launch_overlap_setting_round_trips():
+    before = fv.favor_set_launch_overlap(True)
+    try:
+        assert fv.favor_set_launch_overlap(False) is True
+        assert fv.favor_set_launch_overlap(False) is False
+        assert fv.lib.favor_set_launch_overlap(7) == 0 and fv.lib.favor_set_launch_overlap(0) == 1
+    finally:
+        fv.favor_set_launch_overlap(before)
+
+
 def test_attention_rejects_null_and_misaligned_pointers():
     assert attn([FAKE, 0, FAKE, FAKE, FAKE]) == fv.FAVOR_ERR_INVALID
     assert attn([FAKE, FAKE, FAKE + 8, FAKE, FAKE]) == fv.FAVOR_ERR_INVALID

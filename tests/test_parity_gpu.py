@@ -167,13 +167,22 @@ def test_deterministic_bitwise():
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("overlap", [False, True])
 @pytest.mark.parametrize("H,Hkv,d", [(8, 8, 64), (8, 1, 128)])
-def test_back_to_back_calls_reusing_scratch(H, Hkv, d):
+def test_back_to_back_calls_reusing_scratch(H, Hkv, d, overlap):
     # Three stage sequences issued back to back on one stream with no synchronisation, all
-    # sharing one partial-state and one state buffer.  The kernels are launched so that each
-    # may start while the one before it finishes; each must still wait before it overwrites a
+    # sharing one partial-state and one state buffer.  With launch overlap on, every kernel may
+    # start while the one before it finishes; each must still wait before it overwrites a
     # buffer an earlier kernel reads (the next key pass's partials, the next reduction's state),
     # so every output equals the same call made alone, bit for bit.
+    before = fv.favor_set_launch_overlap(overlap)
+    try:
+        _back_to_back(H, Hkv, d)
+    finally:
+        fv.favor_set_launch_overlap(before)
+
+
+def _back_to_back(H, Hkv, d):
     B, L, m = 2, 8192, 256
     W = fv.favor_make_features(3, m, d).cuda()
     sets = [[t.cuda() for t in wl.random_inputs(B, H, Hkv, L, d, torch.bfloat16, seed=20 + i)] for i in range(3)]
