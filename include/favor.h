@@ -75,11 +75,17 @@ typedef struct CUstream_st* favor_stream_t; /* the same type as cudaStream_t */
  * 1: a programmatic dependent launch, like the later kernels of a call: it may
  * start as soon as the kernel before it on the stream lets its dependents start
  * (griddepcontrol.launch_dependents) or exits, and it reads its inputs (Q, K, V,
- * W, or a stage call's partial state or state) at once.  Enable it only if no
- * kernel placed on a stream before a library call lets its dependents start
- * before its writes are complete; kernels that do not use programmatic
- * dependent launch never do.  A call's set-up then overlaps the end of the
- * kernel before it (for back-to-back calls, the previous query pass).
+ * W, or a stage call's partial state or state) at once, before that kernel's
+ * writes are guaranteed to be visible.  The library's own kernels let their
+ * dependents start at entry.  So with 1, NO INPUT OF A CALL MAY BE WRITTEN BY THE
+ * KERNEL JUST BEFORE IT ON THE STREAM when that kernel is one of this library's
+ * (for example, the out of one call fed as Q, K or V of the next, as in stacked
+ * layers) or any other kernel that lets its dependents start early; chained calls
+ * like these need 0, or an event or any ordinary kernel launch between them.
+ * Kernels that do not use programmatic dependent launch never let dependents
+ * start early, so after them 1 is safe.  A call's set-up then overlaps the end of
+ * the kernel before it (for back-to-back calls on independent inputs, the
+ * previous query pass).
  */
 FAVOR_API int favor_set_launch_overlap(int enable);
 
@@ -222,7 +228,9 @@ FAVOR_API int favor_query_pass(int dtype, const void* Q, const float* W, const v
  * favor_last_error().  Every call shares the one array and overwrites all of
  * the scratch it uses, so nothing has to be cleared between calls, but calls
  * that overlap on the GPU (on different streams, or from different threads)
- * race on it: serialise them.
+ * race on it: serialise them.  The looked-up address belongs to the device's
+ * primary context of the process: after cudaDeviceReset (or any teardown of that
+ * context) this entry point must not be called again in the same process.
  */
 FAVOR_API int favor_attention_noalloc(int dtype, const void* Q, const void* K, const void* V, const float* W,
                                       void* out, int B, int H, int Hkv, int L, int d, int m,

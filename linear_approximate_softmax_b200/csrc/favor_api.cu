@@ -118,8 +118,9 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
   p->st_S_off = 0;
   p->st_c_off = round_up(sizeof(float) * heads * m * D1, 256);
   p->st_op_off = p->st_c_off + round_up(sizeof(float) * heads, 256);
-  // the query pass's state operand: d rows of fp16 (the normaliser column goes to the tail)
-  p->op_rows = d;
+  // the query pass's state operand: d rows of fp16, and for d = 64 the normaliser as row d and 15
+  // rows of zeros (the tensor-core query pass reads them as 16 more output columns)
+  p->op_rows = d == 64 ? d + 16 : d;
   p->op_atoms = (m + 63) / 64;
   p->op_tail = (m + 127) / 128 * 128;
   // fp16 rows (64 features per 128-byte row), then one fp32 exponent per feature, then the

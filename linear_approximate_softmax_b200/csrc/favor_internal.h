@@ -32,8 +32,9 @@ struct Plan {
   // byte offsets inside the state buffer
   size_t st_S_off, st_c_off, st_op_off, st_bytes;
   // The state re-packed as the fp16 B operand of the query pass's second MMA.
-  // Per kv head: op_atoms blocks of 64 features, each op_rows = d rows (output
-  // column n) of 128 B, K-major with the 128-byte swizzle (16-byte chunk c of row n
+  // Per kv head: op_atoms blocks of 64 features, each op_rows rows (output column n; for
+  // d = 64 rows d .. d + 15 follow: the normaliser column, then zeros) of 128 B, K-major
+  // with the 128-byte swizzle (16-byte chunk c of row n
   // at c ^ (n % 8)); then e[op_tail] and the normaliser column s[op_tail], fp32, with
   // op_tail = m rounded up to 128.  Feature f's values are 2^-x_f S[f][n] relative to
   // its own largest chunk stabiliser c_f, with x_f chosen so that the largest lands in

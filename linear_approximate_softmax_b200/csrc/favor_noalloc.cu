@@ -74,6 +74,8 @@ extern "C" int favor_attention_noalloc(int dtype, const void* Q, const void* K, 
     const size_t room = kStaticScratchBytes - st_room;
     plan_limit_chunks(&p, static_cast<int>(room / per_chunk));
   }
+  // the estimate above ignores the 256-byte rounding of each array: step down until it fits
+  while (round256(p.part_bytes) + p.st_bytes > kStaticScratchBytes && p.P > 1) plan_limit_chunks(&p, p.P - 1);
   const size_t st_off = round256(p.part_bytes);
   if (st_off + p.st_bytes > kStaticScratchBytes)
     return set_errorf(FAVOR_ERR_UNSUPPORTED,

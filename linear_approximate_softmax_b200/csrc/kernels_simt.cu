@@ -168,12 +168,14 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel(
     const float* __restrict__ part_S, const float* __restrict__ part_c, float* __restrict__ S,
     float* __restrict__ Sc, unsigned char* __restrict__ op, int P, int m, int nsb, int op_atoms, int op_tail,
-    size_t op_bytes) {
+    size_t op_bytes, int op_rows) {
   constexpr int D1 = D + 1;
   constexpr int NC = (D1 + 7) / 8;     // columns per thread: g, g + 8, ...
   constexpr int CB = D == 64 ? 3 : 2;  // chunks whose rows are in flight together
   __shared__ float red[kThreads / 32];
-  __shared__ __align__(16) __half stage[D][32];  // the image rows of this CTA's 32 features
+  // the image rows of this CTA's 32 features: D outputs, then (when the image has D + 16 rows)
+  // the normaliser row and 15 rows of zeros
+  __shared__ __align__(16) __half stage[D + 16][32];
   griddep_launch_dependents();
   griddep_wait();  // the partial state comes from the kernel before this one on the stream
   const int head = blockIdx.y, tid = threadIdx.x;
@@ -228,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
   for (int k = 0; k < NC; ++k) {
     const int n = g + 8 * k;
     if (live && n < D1) S[(static_cast<size_t>(head) * m + f) * D1 + n] = val[k] * rel;
-    if (n < D) amax = fmaxf(amax, fabsf(val[k]));
+    if (n <= D) amax = fmaxf(amax, fabsf(val[k]));  // the normaliser must fit fp16 too
     if (n == D) den = val[k];
   }
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
@@ -248,11 +250,13 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
 #pragma unroll
   for (int k = 0; k < NC; ++k) {
     const int n = g + 8 * k;
-    if (n < D) stage[n][fl] = __float2half_rn(val[k] * sa * sb);
+    if (n <= D) stage[n][fl] = __float2half_rn(val[k] * sa * sb);
   }
+  stage[D + 1 + g][fl] = __float2half_rn(0.f);              // rows D+1 .. D+8
+  if (g < 7) stage[D + 9 + g][fl] = __float2half_rn(0.f);  // rows D+9 .. D+15
   unsigned char* img = op + static_cast<size_t>(head) * op_bytes;
   // tail: the exponent of each feature, then its normaliser entry with the same scaling
-  float* tail = reinterpret_cast<float*>(img + static_cast<size_t>(D) * 128 * op_atoms);
+  float* tail = reinterpret_cast<float*>(img + static_cast<size_t>(op_rows) * 128 * op_atoms);
   if (g == 0) tail[f] = live && cf > -INFINITY ? static_cast<float>(ex) + (cf - cs) : -INFINITY;
   if ((D & 7) == g) tail[op_tail + f] = live ? den * sa * sb : 0.f;
   __syncthreads();
@@ -260,9 +264,9 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
   // this CTA's 32 features are four chunks of each row of its 64-feature atom
   const int atom = f0 >> 6;
   if (atom < op_atoms)
-    for (int i = tid; i < D * 4; i += kThreads) {
+    for (int i = tid; i < op_rows * 4; i += kThreads) {
       const int n = i >> 2, c4 = i & 3, chunk = ((f0 & 63) >> 3) + c4;
-      const size_t off = static_cast<size_t>(atom) * D * 128 + static_cast<size_t>(n) * 128 + ((chunk ^ (n & 7)) << 4);
+      const size_t off = static_cast<size_t>(atom) * op_rows * 128 + static_cast<size_t>(n) * 128 + ((chunk ^ (n & 7)) << 4);
       *reinterpret_cast<uint4*>(img + off) = *reinterpret_cast<const uint4*>(&stage[n][8 * c4]);
     }
 }
@@ -404,7 +408,7 @@ int simt_state_reduce(const void* partials, void* state, const Plan& p, void* st
       kern, grid, dim3(kThreads), 0, st, overlap, reinterpret_cast<const float*>(pb + p.part_S_off),
       reinterpret_cast<const float*>(pb + p.part_c_off), reinterpret_cast<float*>(sb + p.st_S_off),
       reinterpret_cast<float*>(sb + p.st_c_off), reinterpret_cast<unsigned char*>(sb + p.st_op_off), p.P, p.m, p.nsb,
-      p.op_atoms, p.op_tail, p.op_bytes);
+      p.op_atoms, p.op_tail, p.op_bytes, p.op_rows);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "state reduce launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
 }

@@ -806,6 +806,7 @@ struct QueryCfg {
                        B_OE = 16, B_SF = 18, B_SE = 19, B_STG = 20, NBAR = 24;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
+  static constexpr int S_IMGS = S_ABORT + 4;  // state images loaded so far (published by warp 3)
   static constexpr int SMEM = S_ABORT + 16 + 1024;
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(S_SP % 1024 == 0 && S_Q % 1024 == 0 && S_STG % 1024 == 0, "128-byte swizzled operands start on 1024-byte boundaries");
@@ -850,6 +851,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   // so the CTA's tiles visit each kv head once: image index 0 .. nimg - 1
   const int kvh0 = T0 / ntq / G;
   const int nimg = n > 0 ? (T0 + n - 1) / ntq / G - kvh0 + 1 : 0;
+  int* img_count = reinterpret_cast<int*>(smem + C::S_IMGS);
 
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -867,6 +869,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     mbar_init(bar(C::B_SE), 2);  // an image is released once both issuers are done with it
     for (int i = 0; i < 4; ++i) mbar_init(bar(C::B_STG + i), 1);
     *abort_flag = 0;
+    *img_count = 0;
     fence_barrier_init();
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmO);
@@ -924,9 +927,9 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   if (warp < C::EPI0) {
   setmaxnreg_dec<kRegsLow>();
   if (warp == 0) {
-    // ---------------- producer: Q tiles (stage = tile parity) and state images ----------------
+    // ---------------- producer: Q tiles (stage = tile parity) ----------------
     if (lane == 0) {
-      int loaded = n > 0 ? 0 : -1, issued = 0;  // tiles 0 and 1 and image 0 were issued during the set-up
+      int issued = 0;  // tiles 0 and 1 were issued during the set-up
       TileCursor pc;
       pc.init(T0, ntq, G, kvh0);
       for (int it = 0; it < n; ++it, pc.step(1, ntq, G)) {
@@ -940,17 +943,30 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
                         pc.bh);
         }
         issued = it + 1;
-        const int k = pc.img;
-        if (k > loaded) {  // a new kv head: load its image once both issuers have released the previous one
-          if (k >= 1 && !mbar_wait(bar(C::B_SE), (k - 1) & 1, abort_flag, err)) break;
-          mbar_arrive_expect_tx(bar(C::B_SF), op_bytes);
-          bulk_load(sbase + C::S_SP, op_img + static_cast<size_t>(kvh0 + k) * op_bytes, op_bytes, bar(C::B_SF));
-          loaded = k;
-        }
       }
       for (int it = max(0, issued - 2); it < issued; ++it)
         mbar_wait(bar(C::B_QF + (it & 1)), (it >> 1) & 1, abort_flag, err, 200000000ull);
-      if (loaded >= 0) mbar_wait(bar(C::B_SF), loaded & 1, abort_flag, err, 200000000ull);
+    }
+  } else if (warp == 3) {
+    // ---------------- state images: image k once both issuers have released image k - 1 ----------------
+    // The image warp is the only waiter on SF, so it waits its phases in order, and publishes a count
+    // of loaded images: a warpgroup whose tiles skip a kv head cannot mistake an earlier phase of the
+    // same parity for its image.
+    if (lane == 0 && n > 0) {
+      int k = 0;
+      bool inflight = true;  // image 0, issued during the set-up
+      for (; k < nimg; ++k) {
+        if (k >= 1) {
+          if (!mbar_wait<true>(bar(C::B_SE), (k - 1) & 1, abort_flag, err)) break;
+          mbar_arrive_expect_tx(bar(C::B_SF), op_bytes);
+          bulk_load(sbase + C::S_SP, op_img + static_cast<size_t>(kvh0 + k) * op_bytes, op_bytes, bar(C::B_SF));
+          inflight = true;
+        }
+        if (!mbar_wait<true>(bar(C::B_SF), k & 1, abort_flag, err)) break;
+        inflight = false;
+        st_release_shared(img_count, k + 1);
+      }
+      if (inflight) mbar_wait(bar(C::B_SF), k & 1, abort_flag, err, 200000000ull);  // drain after a failure
     }
   } else if (warp == 1 || warp == 2) {
     // ---------------- MMA issuer of warpgroup w = warp - 1: its tiles w, w + 2, ... ----------------
@@ -1015,7 +1031,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         if (!mbar_wait(bar(C::B_PHI + w), b & 1, abort_flag, err)) break;
         if (j == 0) {
           if (tc >= 1 && !mbar_wait(bar(C::B_OE + w), (tc - 1) & 1, abort_flag, err)) break;
-          if (!mbar_wait(bar(C::B_SF), k & 1, abort_flag, err)) break;
+          if (!wait_count_above(img_count, k, abort_flag, err)) break;
         }
         tc_fence_after();
         const int bw = min(FB, m - FB * j);
@@ -1114,7 +1130,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     if (ewg < n) ec.init(T0 + ewg, ntq, G, kvh0);
     for (int t = ewg; t < n; t += 2, ++tc, ec.step(2, ntq, G)) {
       const float up = up_next;
-      mbar_wait(bar(C::B_SF), ec.img & 1, abort_flag, err);  // this tile's image (exponents) is in
+      wait_count_above(img_count, ec.img, abort_flag, err);  // this tile's image (exponents) is in
       float c = 0.f, den = 0.f;
       for (int j = 0; j < nb; ++j, ++cntb) {
         mbar_wait(bar(C::B_UF + ewg), cntb & 1, abort_flag, err);
@@ -1240,6 +1256,8 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   if (warp == 1) tmem_dealloc(tbase, 512);
 }
 
+#include "query_pass_d64.cuh"
+
 // ============================================================================
 // Host side
 // ============================================================================
@@ -1286,12 +1304,12 @@ int num_sms() {
 // The kernels that rebalance registers between warpgroups (setmaxnreg) need the launch to
 // hold at least what the rebalanced warpgroups ask for, or the increase would never be
 // granted: check the compiled register count once per kernel before the first launch.
-int check_register_split(const void* kern, int threads) {
+int check_register_split(const void* kern, int threads, long need = -1) {
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 kernel attributes: %s", cudaGetErrorString(e));
   const long have = static_cast<long>(fa.numRegs) * threads;
-  const long need = 128L * kRegsLow + static_cast<long>(threads - 128) * kRegsHigh;
+  if (need < 0) need = 128L * kRegsLow + static_cast<long>(threads - 128) * kRegsHigh;
   if (have < need)
     return set_errorf(FAVOR_ERR_UNSUPPORTED, "sm100 kernel compiled with %d registers per thread: %ld < %ld needed",
                       fa.numRegs, have, need);
@@ -1354,11 +1372,37 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   return FAVOR_OK;
 }
 
+int launch_query_d64(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,
+                     bool overlap) {
+  using C = QueryD64;
+  CUtensorMap mq, mo;
+  const int bh = p.B * p.H;
+  int rc = make_map(&mq, Q, C::D, p.L, bh);
+  if (rc == FAVOR_OK) rc = make_map(&mo, out, C::D, p.L, bh, 32);  // stored by each output warp, 32 rows
+  if (rc != FAVOR_OK) return rc;
+  if (p.op_rows != C::NROWS) return set_error(FAVOR_ERR_UNSUPPORTED, "query pass: state image without the normaliser rows");
+  auto kern = query_pass_d64_sm100;
+  const long need = 128L * C::R_CTL + 128L * C::R_CVT + 256L * C::R_EPI;
+  static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), C::THREADS, need);
+  if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), C::THREADS, need);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass attribute: %s", cudaGetErrorString(e));
+  const int ntiles = bh * ((p.L + 127) / 128);
+  const int grid = ntiles < num_sms() ? ntiles : num_sms();
+  const unsigned char* img = static_cast<const unsigned char*>(state) + p.st_op_off;
+  e = launch_overlapped(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, overlap, mq, mo, W, img, p.L, p.m, p.H,
+                        p.Hkv, ntiles, static_cast<int>(p.op_bytes), p.wscale);
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass launch: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
 }  // namespace
 
 bool sm100_key_supported(const Plan& p) { return p.d == 64 || p.d == 128; }
+// d = 64: the three-warpgroup kernel for m > 64 (m <= 64 is one feature block per tile and runs on
+// the CUDA cores); d = 128: the two-warpgroup kernel for m <= 256
 bool sm100_query_supported(const Plan& p) {
-  return (p.d == 64 && p.m <= QueryCfg<64>::MMAX) || (p.d == 128 && p.m <= QueryCfg<128>::MMAX);
+  return (p.d == 64 && p.m > 64 && p.m <= QueryD64::MMAX) || (p.d == 128 && p.m <= QueryCfg<128>::MMAX);
 }
 
 int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st,
@@ -1369,7 +1413,7 @@ int sm100_key_pass(const void* K, const void* V, const float* W, void* partials,
 
 int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,
                      bool overlap) {
-  return p.d == 64 ? launch_query<64>(Q, W, state, out, p, st, overlap)
+  return p.d == 64 ? launch_query_d64(Q, W, state, out, p, st, overlap)
                    : launch_query<128>(Q, W, state, out, p, st, overlap);
 }
 

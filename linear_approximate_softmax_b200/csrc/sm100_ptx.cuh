@@ -88,6 +88,37 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// A counter in shared memory written by one thread with release semantics and read by others
+// with acquire semantics: unlike an mbarrier's phase parity, a monotonic count cannot be
+// mistaken for an earlier value of the same parity by a waiter that skips ahead.
+__device__ __forceinline__ int ld_acquire_shared(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_shared(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+// Waits until *counter > k, bounded like mbar_wait.
+__device__ __forceinline__ bool wait_count_above(const int* counter, int k, volatile int* abort,
+                                                 unsigned int* err_word, uint64_t limit_ns = 2000000000ull) {
+  if (ld_acquire_shared(counter) > k) return true;
+  if (*abort) return false;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_shared(counter) > k) return true;
+    if ((it & 15u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        atomicOr(err_word, FAVOR_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -80,3 +80,55 @@ def test_clock_summary_reports_throttle_and_survives_garbage():
     assert s["samples"] == 1 and s["sm_mhz"] == 1800.0
     assert s["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     assert _sampler([]) == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_kernel_roofline_picks_the_binding_roof():
+    # headline query pass: 4*12*16384 = 786432 query tokens x 256 exponentials = 201.3 M exps;
+    # at 100 us that is 2013.3 Gexp/s against 16 x 148 x 1.965 GHz = 4653.12 Gexp/s
+    w = wl.WORKLOADS["bf16_L16384_heavykeys"]
+    k = bench.kernel_roofline(w, PEAKS, "query_pass", 0.1)
+    assert k["bound"] == "alu" and k["unit"] == "Gexp/s"
+    assert k["achieved"] == pytest.approx(786432 * 256 / 100e-6 / 1e9)
+    assert k["frac"] == pytest.approx(786432 * 256 / 100e-6 / 4653.12e9)
+    # the multi-query query pass (d = 128): 2*128*256 + 2*256*129 = 131584 flop per query token
+    # needs 16*16*8192 * 131584 / 1642.8e12 = 168.0 us of tensor time against 119.9 us of MUFU
+    # time and 2 * 128 * 2 B / 6538 GB/s per token = 164.2 us of HBM time: tensor-bound
+    wq = wl.WORKLOADS["bf16_mqa_L8192_d128"]
+    kq = bench.kernel_roofline(wq, PEAKS, "query_pass", 0.2)
+    assert kq["bound"] == "tensor" and kq["unit"] == "TFLOP/s"
+    assert kq["achieved"] == pytest.approx(2097152 * 131584 / 200e-6 / 1e12)
+    # the reduction moves its scratch bytes: HBM-bound
+    kr = bench.kernel_roofline(w, PEAKS, "state_reduce", 0.01, (6538 * 10, 0))
+    assert kr["bound"] == "hbm" and kr["achieved"] == pytest.approx(6538 * 10 / 10e-6 / 1e9)
+
+
+def test_fp32_workload_uses_the_fma_roof():
+    # fp32 runs on CUDA cores: 128 FMA/clk/SM x 2 flop x 148 SMs x 1.965 GHz = 74.45 TFLOP/s
+    w = wl.WORKLOADS["fp32_L256"]
+    rt = bench.roofline_terms(w, PEAKS)
+    assert rt["t_tensor_us"] == pytest.approx(rt["flops"] / (2 * 128 * 148 * 1.965e9) * 1e6)
+
+
+def test_both_arms_share_the_config_object():
+    w = wl.WORKLOADS["bf16_L131072_m512"]
+    c = bench.config_of(w, 1)
+    assert c["workload"] == "bf16_L131072_m512" and c["m"] == 512 and c["parallelism"] == "replicas x1"
+    assert "l2" in c and c["orthogonal_W"] is True
+
+
+def test_reference_arm_maps_no_library():
+    # the oracle arm must never load the CUDA library: run it in a fresh interpreter and look
+    # for the library in the process's memory map afterwards
+    import subprocess
+    code = ("import runpy, sys; sys.argv = ['bench.py', '--impl', 'reference', '--workload', 'fp32_L256', "
+            "'--steps', '1', '--warmup', '0']; runpy.run_path('bench.py', run_name='__main__'); "
+            "maps = open('/proc/self/maps').read(); "
+            "print('MAPPED' if 'libfavor_b200' in maps else 'CLEAN'); "
+            "print('IMPORTED' if 'linear_approximate_softmax_b200' in sys.modules else 'NOT_IMPORTED')")
+    p = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT, timeout=300,
+                       env=dict(os.environ, OMP_NUM_THREADS="1"))
+    assert p.returncode == 0, p.stderr[-2000:]
+    out = p.stdout.splitlines()
+    assert "CLEAN" in out and "NOT_IMPORTED" in out
+    line = [__import__("json").loads(x) for x in out if x.startswith("{")][0]
+    assert line["impl"] == "reference" and line["cpu_baseline"]["cores"] == os.cpu_count()
