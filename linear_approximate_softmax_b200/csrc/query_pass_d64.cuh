@@ -68,13 +68,6 @@ struct QueryD64 {
   static_assert(S_SP % 1024 == 0 && S_Q % 1024 == 0 && S_STG % 1024 == 0, "swizzled operands on 1024-byte boundaries");
 };
 
-// a >= b ? a : b over three operands (one instruction), free for the compiler to schedule
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, const float* __restrict__ W,
     const unsigned char* __restrict__ op_img, int L, int m, int H, int Hkv, int ntiles_total, int op_bytes,
