@@ -202,6 +202,42 @@ def softmax_attention(Q, K, V):
 
 
 # --------------------------------------------------------------------------
+# Incremental decoding against the FAVOR+ state ("Fast Transformer Decoding:
+# One Write-Head is All You Need", 研究动机与目标 / motivation and 提出的方法 /
+# proposed method: one token at a time, with H query heads sharing one K/V
+# head; here the cached K/V of each head is replaced by its fixed-size state)
+# --------------------------------------------------------------------------
+def decode_outputs(Q, K, V, W):
+    """Outputs of T decoding steps, fp64.
+
+    Q: [B, H, T, d], K, V: [B, Hkv, T, d].  Step t appends key/value t to each
+    kv head's state and answers query t against it: the state after t + 1
+    tokens is S_t = phi(K'[:t+1])^T [V[:t+1] | 1] (key_state of the first t + 1
+    keys, one stabiliser for the whole head, which cancels), and
+    out[:, :, t] = query_output(Q[:, :, t], W, S_t).  Returns [B, H, T, d].
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, T, d = Q.shape
+    Hkv = K.shape[1]
+    G = H // Hkv
+    out = np.empty((B, H, T, d), dtype=np.float64)
+    for b in range(B):
+        for g in range(Hkv):
+            # phi(K') of every key with one stabiliser for the head, then the running sum over
+            # tokens: S_t is the sum of the first t + 1 rank-one terms phi(k_s)[v_s | 1]^T
+            phik, _ = key_features(K[b, g], W)
+            V1 = np.concatenate([V[b, g], np.ones((T, 1))], axis=1)
+            S = np.zeros((W.shape[0], d + 1))
+            for t in range(T):
+                S = S + np.outer(phik[t], V1[t])
+                for h in range(g * G, (g + 1) * G):
+                    out[b, h, t] = query_output(Q[b, h, t:t + 1], W, S)[0]
+    return out
+
+
+# --------------------------------------------------------------------------
 # Error metrics used by every parity test
 # --------------------------------------------------------------------------
 def error_metrics(got, ref):

@@ -136,3 +136,36 @@ def test_error_metrics():
     got = np.array([1.5, -2.0, 0.25, 1.0])
     ma, mr = favor.error_metrics(got, ref)
     assert ma == 0.5 and mr == pytest.approx(0.75 / 4.0)
+
+
+# ---- incremental decoding ("Fast Transformer Decoding: One Write-Head is All You Need") ----
+def test_decode_equals_causal_quadratic_form():
+    # brute force: step t attends to keys 0..t with the explicit weights phi(q_t')^T phi(k_s')
+    Q, K, V = _inputs(1, 4, 2, 9, 16, scale=0.5, seed=21)
+    W = favor.make_features(4, 32, 16)
+    got = favor.decode_outputs(Q, K, V, W)
+    G = 2
+    for h in range(4):
+        phiq, _ = favor.query_features(Q[0, h], W, stabilise=False)
+        phik, _ = favor.key_features(K[0, h // G], W, stabilise=False)
+        A = np.tril(phiq @ phik.T)  # causal: key s <= query t
+        want = (A @ V[0, h // G]) / A.sum(axis=1, keepdims=True)
+        np.testing.assert_allclose(got[0, h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_decode_last_step_equals_bidirectional_attention():
+    # after the last token the state holds every key: the bidirectional estimate for that query
+    Q, K, V = _inputs(2, 2, 1, 12, 16, scale=0.5, seed=22)
+    W = favor.make_features(5, 48, 16)
+    got = favor.decode_outputs(Q, K, V, W)[:, :, -1]
+    want = favor.favor_attention(Q, K, V, W)[:, :, -1]
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_decode_first_step_returns_the_first_value():
+    # one key: every weight is on it, so the output is v_0 whatever the query
+    Q, K, V = _inputs(1, 3, 1, 4, 16, scale=2.0, seed=23)
+    W = favor.make_features(6, 32, 16)
+    got = favor.decode_outputs(Q, K, V, W)
+    for h in range(3):
+        np.testing.assert_allclose(got[0, h, 0], V[0, 0, 0], rtol=1e-12, atol=1e-12)
