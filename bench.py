@@ -390,6 +390,63 @@ def workload_entry(fv, w, dev, gpu_index, peaks, min_steps, orthogonal=True, min
     return entry
 
 
+DECODE = dict(B=16, H=16, Hkv=1, d=128, m=256)  # the multi-query shape, one token per step
+
+
+def decode_entry(fv, dev, peaks, steps=400, graph_steps=100, T=256):
+    """Incremental decoding: microseconds per step (one new token for each of the B sequences, H query
+    heads each) from a resident state, launched one by one and replayed from a CUDA graph, with the
+    state's HBM traffic (read and written once per step) as the roofline."""
+    c = DECODE
+    B, H, Hkv, d, m = c["B"], c["H"], c["Hkv"], c["d"], c["m"]
+    g = torch.Generator("cpu").manual_seed(0)
+    q = torch.randn(T, B, H, d, generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn(T, B, Hkv, d, generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn(T, B, Hkv, d, generator=g).to(torch.bfloat16).to(dev)
+    W = fv.favor_make_features(1, m, d).to(dev)
+    state = torch.empty(fv.favor_decode_state_bytes(B, Hkv, d, m), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+    st = torch.cuda.current_stream(dev)
+    fv.favor_decode_init(state, B, Hkv, d, m, st)
+
+    def step(t):
+        fv.favor_decode_step(q[t % T], k[t % T], v[t % T], W, state, out, st)
+
+    for t in range(20):
+        step(t)
+    fv.favor_device_check()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for t in range(steps):
+        step(t)
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) / steps * 1e3
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=torch.cuda.Stream(dev)):
+        for t in range(graph_steps):
+            fv.favor_decode_step(q[t % T], k[t % T], v[t % T], W, state, out, torch.cuda.current_stream(dev))
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    e0.record(st)
+    for _ in range(4):
+        graph.replay()
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    us_graph = e0.elapsed_time(e1) / (4 * graph_steps) * 1e3
+    fv.favor_device_check()
+    del graph
+    state_bytes = state.numel()
+    io = (B * H * d * 2 + 2 * B * Hkv * d) * 2 + m * d * 4
+    traffic = 2 * state_bytes + io  # the state read and written once, q, k, v, out and W
+    best = min(us, us_graph)
+    ach = traffic / (best * 1e-6) / 1e9
+    return {"workload": "bf16_decode_mqa_d128_m256", **c, "dtype": "bf16", "us_per_step": us, "us_per_step_graph": us_graph,
+            "tokens_per_step": B, "unit": "us per decoded token (all B sequences, H query heads)",
+            "roofline": {"bound": "hbm", "bytes_per_step": traffic, "achieved": ach, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}}
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -496,6 +553,7 @@ def main():
             for orth in wk.orthogonal:
                 entries.append(workload_entry(fv, wk, dev, local, peaks, args.steps or 20, orth))
         line["per_workload"] = entries
+        line["decode"] = decode_entry(fv, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r, heads, dt, threads = oracle_rate(w, 10.0)
         line["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": host_cores(), "blas_threads": threads,

@@ -236,6 +236,48 @@ FAVOR_API int favor_attention_noalloc(int dtype, const void* Q, const void* K, c
                                       void* out, int B, int H, int Hkv, int L, int d, int m,
                                       favor_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Incremental decoding against a cached state.
+ *
+ * "Fast Transformer Decoding: One Write-Head is All You Need" (研究动机与目标 /
+ * motivation, 提出的方法 / proposed method): one token at a time, every step
+ * reads the whole cache of each key/value head, and H query heads may share one
+ * key/value head.  With FAVOR+ the cache of a kv head is its state: a fixed
+ * m x (d + 1) matrix plus one stabiliser per feature, whatever the number of
+ * tokens seen ("Rethinking Attention with Performers", Abstract: linear space).
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of a decode state for B*Hkv kv heads.  Layout per kv head (fp32):
+ *   S [m][d+1]   sum over the tokens seen of 2^(a_t,f - c_f) [v_t | 1], with
+ *                a_t,f = d^-1/4 log2(e) W_f . k_t - d^-1/2 log2(e) |k_t|^2 / 2
+ *   c [m]        the largest a_t,f seen for each feature (-inf before the first token)
+ * so that exp(...) of the method = 2^(a) and S relative to 2^c.
+ * 0 for unsupported shapes (see favor_decode_step). */
+FAVOR_API size_t favor_decode_state_bytes(int B, int Hkv, int d, int m);
+
+/* favor_decode_init — the empty state (S = 0, c = -inf) of B*Hkv kv heads, on `stream`.
+ * state: device, caller-owned, favor_decode_state_bytes(...) bytes, 16-byte aligned. */
+FAVOR_API int favor_decode_init(void* state, int B, int Hkv, int d, int m, favor_stream_t stream);
+
+/*
+ * favor_decode_step — one decoding step for every sequence of the batch.
+ *
+ * Appends key/value k, v [B, Hkv, d] (one token per kv head) to the state, then
+ * answers the queries q [B, H, d] (query head h reads kv head h / (H / Hkv))
+ * against the updated state: out [B, H, d] = FAVOR+ attention of each query over
+ * every token appended so far, including this one.  dtype: FAVOR_BF16 or
+ * FAVOR_F32 for q, k, v and out; W [m, d] fp32 unscaled; state as above, updated
+ * in place (the stabiliser update is exact: c_f is the running maximum and S is
+ * rescaled whenever it rises).  All pointers device, caller-owned, 16-byte
+ * aligned.  Shapes: d in {64, 128}; m a multiple of 16 in [16, 512]; H % Hkv == 0
+ * with at most 64 query heads per kv head.  Each kv head is one cluster of 8 CTAs
+ * on the CUDA cores (fp32 arithmetic throughout).  Asynchronous on `stream`;
+ * calls on one state must be ordered (each reads the state the previous one wrote).
+ */
+FAVOR_API int favor_decode_step(int dtype, const void* q, const void* k, const void* v, const float* W,
+                                void* state, void* out, int B, int H, int Hkv, int d, int m,
+                                favor_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,7 +29,7 @@ EXPORTS = [
     "favor_last_error", "favor_version", "favor_make_features", "favor_attention",
     "favor_attention_f32", "favor_attention_host", "favor_partials_bytes", "favor_state_bytes",
     "favor_key_pass", "favor_state_reduce", "favor_query_pass", "favor_attention_noalloc", "favor_device_check",
-    "favor_set_launch_overlap",
+    "favor_set_launch_overlap", "favor_decode_state_bytes", "favor_decode_init", "favor_decode_step",
 ]
 
 if not os.path.exists(LIB_PATH):
@@ -65,6 +65,12 @@ lib.favor_attention_noalloc.argtypes = [_i] + _ATT
 lib.favor_attention_noalloc.restype = _i
 lib.favor_set_launch_overlap.argtypes = [_i]
 lib.favor_set_launch_overlap.restype = _i
+lib.favor_decode_state_bytes.argtypes = [_i, _i, _i, _i]
+lib.favor_decode_state_bytes.restype = _sz
+lib.favor_decode_init.argtypes = [_p, _i, _i, _i, _i, _p]
+lib.favor_decode_init.restype = _i
+lib.favor_decode_step.argtypes = [_i, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+lib.favor_decode_step.restype = _i
 
 
 def favor_set_launch_overlap(enable):
@@ -198,6 +204,30 @@ def favor_query_pass(Q, W, state, Hkv, out, stream=None):
     B, H, L, d = Q.shape
     _check(lib.favor_query_pass(_dtype_code(Q), _dev(Q, "Q"), _dev(W, "W"), _dev(state, "state"), _dev(out, "out"),
                                 B, H, Hkv, L, d, W.shape[0], _stream(stream)), "favor_query_pass")
+    return out
+
+
+def favor_decode_state_bytes(B, Hkv, d, m):
+    return int(lib.favor_decode_state_bytes(B, Hkv, d, m))
+
+
+def favor_decode_init(state, B, Hkv, d, m, stream=None):
+    """Empty decode state (uint8 CUDA tensor of favor_decode_state_bytes(...) bytes)."""
+    _check(lib.favor_decode_init(_dev(state, "state"), B, Hkv, d, m, _stream(stream)), "favor_decode_init")
+    return state
+
+
+def favor_decode_step(q, k, v, W, state, out=None, stream=None):
+    """One decoding step: q [B, H, d], k, v [B, Hkv, d] device tensors; updates `state` in place."""
+    code = _dtype_code(q)
+    B, H, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, d) or v.shape != k.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError(f"k, v must be [B, Hkv, d] of q's dtype; got {tuple(k.shape)}, {tuple(v.shape)}")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.favor_decode_step(code, _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(W, "W"), _dev(state, "state"),
+                                 _dev(out, "out"), B, H, Hkv, d, W.shape[0], _stream(stream)), "favor_decode_step")
     return out
 
 

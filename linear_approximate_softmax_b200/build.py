@@ -15,7 +15,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfavor_b200.so")
 
-SOURCES = ["favor_api.cu", "favor_features.cpp", "kernels_simt.cu", "kernels_sm100.cu", "favor_noalloc.cu"]
+SOURCES = ["favor_api.cu", "favor_features.cpp", "kernels_simt.cu", "kernels_sm100.cu", "favor_noalloc.cu",
+           "decode_sm100.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC]
 

@@ -114,3 +114,18 @@ def test_valid_call_without_a_device_reports_cuda_error():
     ptr = lambda x: ctypes.c_void_p(x.ctypes.data)  # noqa: E731
     rc = fv.lib.favor_attention_host(fv.FAVOR_BF16, ptr(q), ptr(q), ptr(q), ptr(w), ptr(q.copy()), 1, 1, 1, 16, 64, 64, None)
     assert rc == fv.FAVOR_ERR_CUDA and fv.lib.favor_last_error()
+
+
+def test_decode_state_bytes_and_argument_errors():
+    # per kv head: S [m][d+1] and c [m], fp32
+    assert fv.favor_decode_state_bytes(2, 1, 128, 256) == 2 * 1 * 256 * 130 * 4
+    assert fv.favor_decode_state_bytes(1, 3, 64, 16) == 3 * 16 * 66 * 4
+    assert fv.favor_decode_state_bytes(1, 1, 96, 256) == 0   # unsupported d
+    assert fv.favor_decode_state_bytes(1, 1, 64, 520) == 0   # m above 512
+    p = ctypes.c_void_p(FAKE)
+    lib = fv.lib
+    assert lib.favor_decode_step(7, p, p, p, p, p, p, 1, 2, 2, 64, 128, None) == fv.FAVOR_ERR_INVALID
+    assert lib.favor_decode_step(0, p, p, p, p, p, p, 1, 3, 2, 64, 128, None) == fv.FAVOR_ERR_UNSUPPORTED
+    assert lib.favor_decode_step(0, p, p, p, p, p, p, 1, 65, 1, 64, 128, None) == fv.FAVOR_ERR_UNSUPPORTED
+    assert lib.favor_decode_step(0, None, p, p, p, p, p, 1, 2, 2, 64, 128, None) == fv.FAVOR_ERR_INVALID
+    assert lib.favor_decode_init(ctypes.c_void_p(FAKE + 8), 1, 1, 64, 128, None) == fv.FAVOR_ERR_INVALID
