@@ -1257,7 +1257,6 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
 }
 
 #include "query_pass_d64.cuh"
-#include "key_pass_d64.cuh"
 
 // ============================================================================
 // Host side
@@ -1314,29 +1313,6 @@ int check_register_split(const void* kern, int threads, long need = -1) {
   if (have < need)
     return set_errorf(FAVOR_ERR_UNSUPPORTED, "sm100 kernel compiled with %d registers per thread: %ld < %ld needed",
                       fa.numRegs, have, need);
-  return FAVOR_OK;
-}
-
-int launch_key_d64(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st,
-                   bool overlap) {
-  using C = KeyD64;
-  CUtensorMap mk, mv;
-  const int heads = p.B * p.Hkv;
-  int rc = make_map(&mk, K, C::D, p.L, heads, C::TB);
-  if (rc == FAVOR_OK) rc = make_map(&mv, V, C::D, p.L, heads, C::TB);
-  if (rc != FAVOR_OK) return rc;
-  auto kern = key_pass_d64_sm100;
-  const long need = 128L * C::R_CTL + 128L * C::R_CVT + 256L * C::R_EPI;
-  static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), C::THREADS, need);
-  if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), C::THREADS, need);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass attribute: %s", cudaGetErrorString(e));
-  char* base = static_cast<char*>(partials);
-  dim3 grid((p.m + 127) / 128, p.P, heads);
-  e = launch_overlapped(kern, grid, dim3(C::THREADS), C::SMEM, st, overlap, mk, mv, W,
-                        reinterpret_cast<float*>(base + p.part_S_off), reinterpret_cast<float*>(base + p.part_c_off),
-                        p.L, p.m, p.P, p.chunk, p.nsb, p.wscale, p.nscale);
-  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
 }
 
@@ -1431,7 +1407,7 @@ bool sm100_query_supported(const Plan& p) {
 
 int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st,
                    bool overlap) {
-  return p.d == 64 ? launch_key_d64(K, V, W, partials, p, st, overlap)
+  return p.d == 64 ? launch_key<64>(K, V, W, partials, p, st, overlap)
                    : launch_key<128>(K, V, W, partials, p, st, overlap);
 }
 
