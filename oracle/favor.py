@@ -238,6 +238,74 @@ def decode_outputs(Q, K, V, W):
 
 
 # --------------------------------------------------------------------------
+# Generalised kernelizable attention, f = ReLU ("Rethinking Attention with
+# Performers", Abstract: the method also approximates kernelizable attention
+# other than softmax; 연구 질문 / research questions, RQ5).  The pages name no
+# f; the reading taken here is the plainest one: phi(x) = ReLU(W x') / sqrt(m)
+# with the same x' = d**-0.25 x and the same W, and the same linear-time order
+# of products.  ReLU is positively homogeneous, so the input scaling and the
+# 1/sqrt(m) factor cancel in the ratio; no stabiliser is needed (phi >= 0 and
+# bounded by |W x'|).
+# --------------------------------------------------------------------------
+def relu_features(X, W):
+    """phi(x') = max(W x', 0) / sqrt(m) for every scaled row x' of X ([n, m])."""
+    W = np.asarray(W, dtype=np.float64)
+    return np.maximum(scale_inputs(X) @ W.T, 0.0) / math.sqrt(W.shape[0])
+
+
+def relu_attention(Q, K, V, W):
+    """out = phi(Q') (phi(K')^T [V | 1]) / last column, per kv head, fp64.
+
+    Shapes as in ``favor_attention``.  A query whose features all vanish
+    against every key (denominator 0) has no defined output; the division
+    is left to produce it (inf or nan).
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, L, d = Q.shape
+    Hkv = K.shape[1]
+    assert H % Hkv == 0
+    G = H // Hkv
+    out = np.empty((B, H, L, d), dtype=np.float64)
+    for b in range(B):
+        for g in range(Hkv):
+            phik = relu_features(K[b, g], W)
+            V1 = np.concatenate([V[b, g], np.ones((V.shape[2], 1))], axis=1)
+            S = phik.T @ V1
+            for h in range(g * G, (g + 1) * G):
+                nz = relu_features(Q[b, h], W) @ S
+                out[b, h] = nz[:, :d] / nz[:, d:d + 1]
+    return out
+
+
+def arccos1_attention(Q, K, V):
+    """The attention that relu_attention estimates as m grows with iid N(0, I) rows of W.
+
+    E_w[max(w.x, 0) max(w.y, 0)] = |x| |y| (sin t + (pi - t) cos t) / (2 pi), t the
+    angle between x and y (the order-1 arc-cosine kernel), so the weights are
+    that kernel of the scaled rows, normalised over the keys; computed with the
+    L x L matrix formed.
+    """
+    Q = scale_inputs(Q)
+    K = scale_inputs(K)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, L, d = Q.shape
+    G = H // K.shape[1]
+    out = np.empty((B, H, L, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            q, k = Q[b, h], K[b, h // G]
+            nq = np.sqrt(np.sum(q * q, axis=1))[:, None]
+            nk = np.sqrt(np.sum(k * k, axis=1))[None, :]
+            cos = np.clip((q @ k.T) / (nq * nk), -1.0, 1.0)
+            t = np.arccos(cos)
+            A = nq * nk * (np.sin(t) + (math.pi - t) * cos) / (2 * math.pi)
+            out[b, h] = (A @ V[b, h // G]) / A.sum(axis=1, keepdims=True)
+    return out
+
+
+# --------------------------------------------------------------------------
 # Error metrics used by every parity test
 # --------------------------------------------------------------------------
 def error_metrics(got, ref):

@@ -169,3 +169,66 @@ def test_decode_first_step_returns_the_first_value():
     got = favor.decode_outputs(Q, K, V, W)
     for h in range(3):
         np.testing.assert_allclose(got[0, h, 0], V[0, 0, 0], rtol=1e-12, atol=1e-12)
+
+
+# ---- generalised kernelizable attention with f = ReLU --------------------------------
+# "Rethinking Attention with Performers", Abstract and RQ5: the same linear-time scheme
+# for kernels other than softmax.  Pinned to the explicit L x L form, to the closed-form
+# order-1 arc-cosine kernel the random features estimate, and to invariants of the map.
+def test_relu_linear_order_equals_quadratic_form():
+    Q, K, V = _inputs(1, 4, 2, 40, 16, seed=21)
+    W = favor.make_features(5, 48, 16)
+    G = 2
+    want = np.empty_like(Q)
+    for h in range(4):
+        pq = favor.relu_features(Q[0, h], W)
+        pk = favor.relu_features(K[0, h // G], W)
+        A = pq @ pk.T
+        want[0, h] = (A @ V[0, h // G]) / A.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(favor.relu_attention(Q, K, V, W), want, rtol=1e-11, atol=1e-12)
+
+
+def test_relu_features_estimate_the_arccos_kernel():
+    # E_w[relu(w.x) relu(w.y)] for w ~ N(0, I): the order-1 arc-cosine kernel; checked by
+    # Monte Carlo over many iid draws, with the standard error as the yardstick
+    d = 8
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal(d)
+    y = rng.standard_normal(d)
+    W = favor.make_features(23, 200_000, d, orthogonal=False)
+    prods = np.maximum(W @ x, 0) * np.maximum(W @ y, 0)
+    nx, ny = np.linalg.norm(x), np.linalg.norm(y)
+    t = math.acos(float(x @ y) / (nx * ny))
+    closed = nx * ny * (math.sin(t) + (math.pi - t) * math.cos(t)) / (2 * math.pi)
+    se = prods.std(ddof=1) / math.sqrt(prods.size)
+    assert abs(prods.mean() - closed) < 4 * se, (prods.mean(), closed, se)
+    assert se < 0.01 * closed
+
+
+def test_relu_attention_converges_to_arccos_attention_as_m_grows():
+    Q, K, V = _inputs(1, 1, 1, 24, 16, seed=24)
+    want = favor.arccos1_attention(Q, K, V)
+    errs = []
+    for m in (64, 1024, 16384):
+        W = favor.make_features(25, m, 16, orthogonal=False)
+        errs.append(np.abs(favor.relu_attention(Q, K, V, W) - want).max())
+    assert errs[0] > errs[1] > errs[2], errs
+    assert errs[2] < 0.02, errs
+
+
+def test_relu_attention_is_scale_free_and_convex():
+    Q, K, V = _inputs(1, 2, 1, 30, 16, seed=26)
+    W = favor.make_features(27, 64, 16)
+    out = favor.relu_attention(Q, K, V, W)
+    # positive homogeneity of relu: scaling queries or keys by a > 0 changes nothing
+    np.testing.assert_allclose(favor.relu_attention(3.7 * Q, 0.25 * K, V, W), out, rtol=1e-11, atol=1e-12)
+    lo, hi = V[0, 0].min(axis=0), V[0, 0].max(axis=0)
+    assert np.all(out >= lo - 1e-12) and np.all(out <= hi + 1e-12)
+
+
+def test_relu_attention_with_identical_keys_returns_the_mean_value():
+    Q, K, V = _inputs(1, 1, 1, 20, 16, seed=28)
+    K[:] = K[0, 0, 0]
+    W = favor.make_features(29, 32, 16)
+    out = favor.relu_attention(Q, K, V, W)
+    np.testing.assert_allclose(out[0, 0], np.broadcast_to(V[0, 0].mean(axis=0), (20, 16)), rtol=1e-11, atol=1e-12)
