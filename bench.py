@@ -447,6 +447,51 @@ def decode_entry(fv, dev, peaks, steps=400, graph_steps=100, T=256):
                          "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}}
 
 
+def relu_entry(fv, dev, peaks, min_seconds=0.4):
+    """Kernelizable attention with f = ReLU (favor_attention_relu) on the headline shape: ms per call,
+    with the path's roofline (fp32 FMA flops of both passes on the CUDA cores, or HBM bytes)."""
+    w = wl.WORKLOADS["bf16_L16384_heavykeys"]
+    Q, K, V = (t.to(dev) for t in wl.make_inputs(w))
+    W = fv.favor_make_features(w.w_seed, w.m, w.d).to(dev)
+    set_bytes = (2 * Q.numel() + K.numel() + V.numel()) * Q.element_size()
+    sets = [(Q, K, V, torch.empty_like(Q))]
+    for _ in range(max(1, math.ceil(2 * L2_BYTES / set_bytes)) - 1):
+        sets.append((Q.clone(), K.clone(), V.clone(), torch.empty_like(Q)))
+    st = torch.cuda.current_stream(dev)
+
+    def call(i):
+        q, k, v, o = sets[i % len(sets)]
+        fv.favor_attention_relu(q, k, v, W, o, st)
+
+    for i in range(3):
+        call(i)
+    fv.favor_device_check()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    call(0)
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    steps = max(5, math.ceil(min_seconds * 1e3 / max(e0.elapsed_time(e1), 1e-3)))
+    e0.record(st)
+    for i in range(steps):
+        call(i)
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    fv.favor_device_check()
+    ms = e0.elapsed_time(e1) / steps
+    G = w.H // w.Hkv
+    flops = w.units * (1 + 1 / G) * (2 * w.d * w.m + 2 * w.m * (w.d + 1))
+    hbm = w.units * 2 * (2 * w.d + 2 * w.d / G)
+    fma_pk = 2 * FFMA_PER_SM_CLK * NUM_SMS * peaks["sm_max_mhz"] * 1e6
+    t = {"fma": flops / fma_pk * 1e6, "hbm": hbm / (peaks["hbm_gbs"] * 1e9) * 1e6}
+    bound = max(t, key=t.get)
+    return {"workload": w.name + "_relu", "feature_map": "relu", "dtype": "bf16", "steps": steps, "ms_per_step": ms,
+            "value": whole_job_rate(w.units, 1, ms), "unit": UNIT,
+            "roofline_path": {"t_fma_us": t["fma"], "t_hbm_us": t["hbm"], "bound": bound,
+                              "frac": t[bound] / (ms * 1e3)},
+            "input_sets": len(sets)}
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -554,6 +599,7 @@ def main():
                 entries.append(workload_entry(fv, wk, dev, local, peaks, args.steps or 20, orth))
         line["per_workload"] = entries
         line["decode"] = decode_entry(fv, dev, peaks)
+        line["relu"] = relu_entry(fv, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r, heads, dt, threads = oracle_rate(w, 10.0)
         line["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": host_cores(), "blas_threads": threads,

@@ -151,6 +151,24 @@ FAVOR_API int favor_attention_f32(const float* Q, const float* K, const float* V
                         int B, int H, int Hkv, int L, int d, int m, favor_stream_t stream);
 
 /*
+ * favor_attention_relu — generalised kernelizable attention with f = ReLU.
+ *
+ * "Rethinking Attention with Performers" (Abstract; 연구 질문 / research
+ * questions, RQ5): the same linear-time scheme approximates attention with
+ * kernels other than softmax.  The pages name no f; this is the plainest one:
+ * phi(x) = max(W x', 0) / sqrt(m), x' = d^-1/4 x, with the same W, and
+ * out = phi(Q')(phi(K')^T V) / (phi(Q')(phi(K')^T 1)).  The scalings cancel in
+ * the ratio (ReLU is positively homogeneous) and no stabiliser is needed.
+ * dtype FAVOR_BF16 or FAVOR_F32 for Q, K, V and out; arguments, layouts,
+ * shapes, scratch and errors as favor_attention.  It runs on the CUDA cores in
+ * fp32 (key pass per chunk, the fixed-order reduction, query pass).  A query
+ * whose features meet no key's (denominator 0) gets inf or nan, as the
+ * division gives.
+ */
+FAVOR_API int favor_attention_relu(int dtype, const void* Q, const void* K, const void* V, const float* W,
+                         void* out, int B, int H, int Hkv, int L, int d, int m, favor_stream_t stream);
+
+/*
  * favor_attention_host — end-to-end call on HOST buffers.
  *
  * Q, K, V, out are host pointers (pinned memory gives asynchronous copies;

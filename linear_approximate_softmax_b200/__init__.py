@@ -30,6 +30,7 @@ EXPORTS = [
     "favor_attention_f32", "favor_attention_host", "favor_partials_bytes", "favor_state_bytes",
     "favor_key_pass", "favor_state_reduce", "favor_query_pass", "favor_attention_noalloc", "favor_device_check",
     "favor_set_launch_overlap", "favor_decode_state_bytes", "favor_decode_init", "favor_decode_step",
+    "favor_attention_relu",
 ]
 
 if not os.path.exists(LIB_PATH):
@@ -49,6 +50,8 @@ lib.favor_attention_f32.argtypes = _ATT
 lib.favor_attention_f32.restype = _i
 lib.favor_attention_host.argtypes = [_i] + _ATT
 lib.favor_attention_host.restype = _i
+lib.favor_attention_relu.argtypes = [_i] + _ATT
+lib.favor_attention_relu.restype = _i
 lib.favor_partials_bytes.argtypes = [_i, _i, _i, _i, _i]
 lib.favor_partials_bytes.restype = _sz
 lib.favor_state_bytes.argtypes = [_i, _i, _i, _i]
@@ -151,6 +154,19 @@ def favor_attention(Q, K, V, W, out=None, stream=None):
 
 
 favor_attention_f32 = favor_attention
+
+
+def favor_attention_relu(Q, K, V, W, out=None, stream=None):
+    """Kernelizable attention with phi = ReLU(W x') on device tensors; bf16 or fp32."""
+    code = _dtype_code(Q)
+    if K.dtype != Q.dtype or V.dtype != Q.dtype or W.dtype != torch.float32:
+        raise TypeError("Q, K, V must share a dtype and W must be float32")
+    B, H, Hkv, L, d, m = _shape(Q, K, V, W)
+    if out is None:
+        out = torch.empty_like(Q)
+    _check(lib.favor_attention_relu(code, _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(W, "W"), _dev(out, "out"),
+                                    B, H, Hkv, L, d, m, _stream(stream)), "favor_attention_relu")
+    return out
 
 
 def favor_attention_host(Q, K, V, W, out=None, stream=None):

@@ -222,6 +222,28 @@ int attention_impl(int dtype, const void* Q, const void* K, const void* V, const
   return FAVOR_OK;
 }
 
+// phi = ReLU(W x'): the same plan and scratch, the CUDA-core key and query passes with the
+// ReLU map, the shared reduction.
+int relu_attention_impl(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,
+                        int H, int Hkv, int L, int d, int m, cudaStream_t st) {
+  FAVOR_TRY(check_dtype(dtype));
+  FAVOR_TRY(check_ptrs("favor_attention_relu", {Q, K, V, W, out}));
+  Plan p;
+  FAVOR_TRY(make_plan(B, H, Hkv, L, d, m, &p));
+  keep_pool_mapped();
+  void* ws = nullptr;
+  const size_t st_off = round_up(p.part_bytes, 256);
+  FAVOR_CUDA_TRY(cudaMallocAsync(&ws, st_off + p.st_bytes, st), "favor_attention_relu scratch allocation");
+  char* base = static_cast<char*>(ws);
+  int rc = simt_key_pass_relu(dtype, K, V, W, base, p, st);
+  if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, p, st, false);
+  if (rc == FAVOR_OK) rc = simt_query_pass_relu(dtype, Q, W, base + st_off, out, p, st);
+  cudaError_t fe = cudaFreeAsync(ws, st);
+  if (rc != FAVOR_OK) return rc;
+  FAVOR_CUDA_TRY(fe, "favor_attention_relu scratch release");
+  return FAVOR_OK;
+}
+
 }  // namespace
 }  // namespace favor
 
@@ -249,6 +271,11 @@ int favor_attention(const void* Q, const void* K, const void* V, const float* W,
 int favor_attention_f32(const float* Q, const float* K, const float* V, const float* W, float* out, int B, int H,
                         int Hkv, int L, int d, int m, favor_stream_t stream) {
   return attention_impl(FAVOR_F32, Q, K, V, W, out, B, H, Hkv, L, d, m, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int favor_attention_relu(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,
+                         int H, int Hkv, int L, int d, int m, favor_stream_t stream) {
+  return relu_attention_impl(dtype, Q, K, V, W, out, B, H, Hkv, L, d, m, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int favor_attention_host(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,

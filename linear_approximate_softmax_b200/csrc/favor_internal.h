@@ -72,6 +72,12 @@ int simt_key_pass(int dtype, const void* K, const void* V, const float* W, void*
 int simt_state_reduce(const void* partials, void* state, const Plan& p, void* stream, bool overlap);
 int simt_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out,
                     const Plan& p, void* stream);
+// The same key and query passes with the feature map f = ReLU (no stabilisers); the
+// reduction is shared.
+int simt_key_pass_relu(int dtype, const void* K, const void* V, const float* W, void* partials, const Plan& p,
+                       void* stream);
+int simt_query_pass_relu(int dtype, const void* Q, const float* W, const void* state, void* out, const Plan& p,
+                         void* stream);
 
 // ---- tensor-core kernels (sm_100a, bf16 storage) ------------------------------
 bool sm100_key_supported(const Plan& p);

@@ -17,6 +17,11 @@
 // = exp(W k' - |k'|^2/2) with k' = d^-1/4 k.  The query's -|q'|^2/2 term and
 // the 1/sqrt(m) factors are constant along a query row and cancel exactly in
 // the ratio, as any per-row stabiliser does; they are not computed.
+//
+// The key and query kernels also serve the generalised kernelizable attention
+// of the same page (Abstract; 연구 질문 RQ5) with f = ReLU: phi = max(W'x, 0) with
+// W' = d^-1/4 W, no norm term and no stabiliser (phi >= 0 is bounded by |W'x|; the
+// chunk stabilisers are written as 0, so the reduction sums the chunks as they are).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -33,6 +38,8 @@ constexpr int kThreads = 256;
 constexpr int kFB = 64;   // features per key-pass CTA
 constexpr int kTT = 32;   // tokens per key-pass step
 constexpr int kQT = 32;   // queries per query-pass CTA
+constexpr int kExp = 0;   // feature maps: FAVOR+ positive features (exp)
+constexpr int kRelu = 1;  //               max(W'x, 0)
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -46,8 +53,8 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // grid (P, B*Hkv, ceil(m/64)), 256 threads.  One running stabiliser per CTA,
-// written for each of its features.
-template <typename T, int D>
+// written for each of its features (0 for f = ReLU).
+template <typename T, int D, int FMAP>
 __global__ void __launch_bounds__(kThreads) key_pass_kernel(
     const T* __restrict__ K, const T* __restrict__ V, const float* __restrict__ W,
     float* __restrict__ part_S, float* __restrict__ part_c, int L, int m, int P, int chunk,
@@ -95,7 +102,8 @@ __global__ void __launch_bounds__(kThreads) key_pass_kernel(
     __syncthreads();
     if (tid < kTT) {
       float s = 0.f;
-      for (int j = 0; j < D; ++j) s = fmaf(Ks[tid * D1 + j], Ks[tid * D1 + j], s);
+      if (FMAP == kExp)
+        for (int j = 0; j < D; ++j) s = fmaf(Ks[tid * D1 + j], Ks[tid * D1 + j], s);
       Ks[tid * D1 + D] = s * nscale;
     }
     __syncthreads();
@@ -113,19 +121,24 @@ __global__ void __launch_bounds__(kThreads) key_pass_kernel(
       U[t * (kFB + 1) + f] = u;
       lmax = fmaxf(lmax, u);
     }
-    lmax = warp_max(lmax);
-    if (lane == 0) red[warp] = lmax;
-    __syncthreads();
-    float tmax = red[0];
+    float rescale = 1.f;
+    if (FMAP == kExp) {
+      lmax = warp_max(lmax);
+      if (lane == 0) red[warp] = lmax;
+      __syncthreads();
+      float tmax = red[0];
 #pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) tmax = fmaxf(tmax, red[w]);
-    const float c_new = fmaxf(c_run, tmax);
-    const float rescale = (c_run == -INFINITY) ? 1.f : exp2f(c_run - c_new);
-    c_run = c_new;
+      for (int w = 1; w < kThreads / 32; ++w) tmax = fmaxf(tmax, red[w]);
+      const float c_new = fmaxf(c_run, tmax);
+      rescale = (c_run == -INFINITY) ? 1.f : exp2f(c_run - c_new);
+      c_run = c_new;
+    } else {
+      c_run = 0.f;
+    }
     for (int i = tid; i < kTT * kFB; i += kThreads) {
       const int t = i / kFB, f = i % kFB;
       const float u = U[t * (kFB + 1) + f];
-      U[t * (kFB + 1) + f] = (u == -INFINITY) ? 0.f : exp2f(u - c_new);
+      U[t * (kFB + 1) + f] = FMAP == kExp ? ((u == -INFINITY) ? 0.f : exp2f(u - c_run)) : fmaxf(u, 0.f);
     }
     __syncthreads();
 #pragma unroll
@@ -149,6 +162,7 @@ __global__ void __launch_bounds__(kThreads) key_pass_kernel(
       if (f < fbw) out[static_cast<size_t>(f0 + f) * D1 + c] = acc[k];
     }
   }
+  if (FMAP == kRelu) c_run = 0.f;  // no token in this chunk: still no stabiliser
   for (int f = tid; f < fbw; f += kThreads) part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + f] = c_run;
 }
 
@@ -272,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
 }
 
 // grid (ceil(L/32), B*H), 256 threads.
-template <typename T, int D>
+template <typename T, int D, int FMAP>
 __global__ void __launch_bounds__(kThreads) query_pass_kernel(
     const T* __restrict__ Q, const float* __restrict__ W, const float* __restrict__ S,
     T* __restrict__ out, int L, int m, int H, int Hkv, float wscale) {
@@ -317,11 +331,15 @@ __global__ void __launch_bounds__(kThreads) query_pass_kernel(
   __syncthreads();
   {  // per-row max over the m features, then phi in place; 8 threads per row
     const int r = tid >> 3, k = tid & 7;
-    float mx = -INFINITY;
-    for (int f = k; f < m; f += 8) mx = fmaxf(mx, U[r * mp + f]);
+    if (FMAP == kExp) {
+      float mx = -INFINITY;
+      for (int f = k; f < m; f += 8) mx = fmaxf(mx, U[r * mp + f]);
 #pragma unroll
-    for (int o = 4; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    for (int f = k; f < m; f += 8) U[r * mp + f] = exp2f(U[r * mp + f] - mx);
+      for (int o = 4; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      for (int f = k; f < m; f += 8) U[r * mp + f] = exp2f(U[r * mp + f] - mx);
+    } else {
+      for (int f = k; f < m; f += 8) U[r * mp + f] = fmaxf(U[r * mp + f], 0.f);
+    }
   }
   __syncthreads();
   float acc[NE];
@@ -350,12 +368,16 @@ __global__ void __launch_bounds__(kThreads) query_pass_kernel(
   }
 }
 
-template <typename T, int D>
+// d^-1/4: the input scaling of the ReLU map (no log2(e): no exponential)
+float relu_wscale(int d) { return static_cast<float>(std::pow(static_cast<double>(d), -0.25)); }
+
+template <typename T, int D, int FMAP = kExp>
 int launch_key(const void* K, const void* V, const float* W, void* partials, const Plan& p,
                cudaStream_t st) {
   constexpr int D1 = D + 1;
   const size_t smem = sizeof(float) * (kFB * D1 + 2 * kTT * D1 + kTT * (kFB + 1) + kThreads / 32);
-  auto kern = key_pass_kernel<T, D>;
+  auto kern = key_pass_kernel<T, D, FMAP>;
+  const float wscale = FMAP == kExp ? p.wscale : relu_wscale(p.d);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "key pass attribute: %s", cudaGetErrorString(e));
   dim3 grid(p.P, p.B * p.Hkv, (p.m + kFB - 1) / kFB);
@@ -363,25 +385,26 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(K), static_cast<const T*>(V), W,
                                      reinterpret_cast<float*>(base + p.part_S_off),
                                      reinterpret_cast<float*>(base + p.part_c_off), p.L, p.m, p.P,
-                                     p.chunk, p.nsb, p.wscale, p.nscale);
+                                     p.chunk, p.nsb, wscale, p.nscale);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "key pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
 }
 
-template <typename T, int D>
+template <typename T, int D, int FMAP = kExp>
 int launch_query(const void* Q, const float* W, const void* state, void* out, const Plan& p,
                  cudaStream_t st) {
   constexpr int D1 = D + 1;
   const size_t smem = sizeof(float) * (kQT * D1 + kFB * D1 + kQT * (D1 + 1) + kQT * (p.m + 1));
-  auto kern = query_pass_kernel<T, D>;
+  auto kern = query_pass_kernel<T, D, FMAP>;
+  const float wscale = FMAP == kExp ? p.wscale : relu_wscale(p.d);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "query pass attribute: %s", cudaGetErrorString(e));
   dim3 grid((p.L + kQT - 1) / kQT, p.B * p.H);
   const char* base = static_cast<const char*>(state);
   kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(Q), W,
                                      reinterpret_cast<const float*>(base + p.st_S_off),
-                                     static_cast<T*>(out), p.L, p.m, p.H, p.Hkv, p.wscale);
+                                     static_cast<T*>(out), p.L, p.m, p.H, p.Hkv, wscale);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "query pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
@@ -411,6 +434,26 @@ int simt_state_reduce(const void* partials, void* state, const Plan& p, void* st
       p.op_atoms, p.op_tail, p.op_bytes, p.op_rows);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "state reduce launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
+}
+
+int simt_key_pass_relu(int dtype, const void* K, const void* V, const float* W, void* partials, const Plan& p,
+                       void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FAVOR_F32)
+    return p.d == 64 ? launch_key<float, 64, kRelu>(K, V, W, partials, p, st)
+                     : launch_key<float, 128, kRelu>(K, V, W, partials, p, st);
+  return p.d == 64 ? launch_key<__nv_bfloat16, 64, kRelu>(K, V, W, partials, p, st)
+                   : launch_key<__nv_bfloat16, 128, kRelu>(K, V, W, partials, p, st);
+}
+
+int simt_query_pass_relu(int dtype, const void* Q, const float* W, const void* state, void* out, const Plan& p,
+                         void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FAVOR_F32)
+    return p.d == 64 ? launch_query<float, 64, kRelu>(Q, W, state, out, p, st)
+                     : launch_query<float, 128, kRelu>(Q, W, state, out, p, st);
+  return p.d == 64 ? launch_query<__nv_bfloat16, 64, kRelu>(Q, W, state, out, p, st)
+                   : launch_query<__nv_bfloat16, 128, kRelu>(Q, W, state, out, p, st);
 }
 
 int simt_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out,

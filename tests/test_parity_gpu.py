@@ -125,6 +125,33 @@ def test_query_stabiliser_raised_in_second_feature_block_bf16():
     run_case(Q.bfloat16(), K.bfloat16(), V.bfloat16(), m, what="late queries")
 
 
+def test_scaled_query_rows_take_the_unfolded_path():
+    # A query row whose largest |q| reaches 2^15 overflows fp16 as a projection operand, so it is
+    # scaled by 2^-k, and every row of its 32-row group adds e_f on the CUDA cores instead of
+    # through the projection.  The ordinary rows of such groups must still match the oracle; the
+    # huge rows (whose exponents no fp16 projection resolves) must stay finite and inside the
+    # per-column range of V, since every FAVOR+ weight is positive.
+    d, m, L = 64, 256, 300
+    g = torch.Generator().manual_seed(9)
+    Q = torch.randn(1, 2, L, d, generator=g) * 0.5
+    huge = [5, 40, 77, 130, 261]  # rows in four different 32-row groups and two 128-row tiles
+    for i in huge:
+        u = torch.randn(d, generator=g)
+        Q[0, :, i] = 65536.0 * u / u.abs().max()
+    K = torch.randn(1, 1, L, d, generator=g)
+    V = torch.randn(1, 1, L, d, generator=g)
+    Qb, Kb, Vb = Q.bfloat16(), K.bfloat16(), V.bfloat16()
+    W = fv.favor_make_features(1, m, d)
+    got = f64(gpu_attention(Qb, Kb, Vb, W))
+    assert np.all(np.isfinite(got))
+    ref = ofv.favor_attention(f64(Qb), f64(Kb), f64(Vb), ofv.make_features_f32(1, m, d))
+    normal = np.setdiff1d(np.arange(L), huge)
+    assert_close(got[:, :, normal], ref[:, :, normal], torch.bfloat16, "rows beside scaled rows")
+    v = f64(Vb)[0, 0]
+    lo, hi = v.min(axis=0) - 1e-2, v.max(axis=0) + 1e-2
+    assert np.all((got[0, :, huge] >= lo) & (got[0, :, huge] <= hi))
+
+
 # ---- full sizes, in the launch configuration bench.py times ----------------
 def _bench_path(Qd, Kd, Vd, Wd):
     """The three stage calls back to back with launch overlap on, as bench.py times them."""
