@@ -492,6 +492,56 @@ def relu_entry(fv, dev, peaks, min_seconds=0.4):
             "input_sets": len(sets)}
 
 
+def linformer_entry(fv, dev, peaks, kp=256, min_seconds=0.4):
+    """Linformer projected attention (favor_linformer) on the headline shape with k = 256 projected
+    rows: ms per call, with the path's roofline (fp32 FMA flops of the projections and the attention
+    over k, MUFU exponentials, or HBM bytes of Q, K, V, out, E and F)."""
+    w = wl.WORKLOADS["bf16_L16384_heavykeys"]
+    Q, K, V = (t.to(dev) for t in wl.make_inputs(w))
+    g = torch.Generator("cpu").manual_seed(5)
+    E = (torch.randn(kp, w.L, generator=g) / math.sqrt(w.L)).to(dev)
+    F = (torch.randn(kp, w.L, generator=g) / math.sqrt(w.L)).to(dev)
+    set_bytes = (2 * Q.numel() + K.numel() + V.numel()) * Q.element_size()
+    sets = [(Q, K, V, torch.empty_like(Q))]
+    for _ in range(max(1, math.ceil(2 * L2_BYTES / set_bytes)) - 1):
+        sets.append((Q.clone(), K.clone(), V.clone(), torch.empty_like(Q)))
+    st = torch.cuda.current_stream(dev)
+
+    def call(i):
+        q, k, v, o = sets[i % len(sets)]
+        fv.favor_linformer(q, k, v, E, F, o, st)
+
+    for i in range(3):
+        call(i)
+    fv.favor_device_check()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    call(0)
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    steps = max(5, math.ceil(min_seconds * 1e3 / max(e0.elapsed_time(e1), 1e-3)))
+    e0.record(st)
+    for i in range(steps):
+        call(i)
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    fv.favor_device_check()
+    ms = e0.elapsed_time(e1) / steps
+    kv_heads, q_heads = w.B * w.Hkv, w.B * w.H
+    flops = kv_heads * 2 * (2 * kp * w.L * w.d) + q_heads * w.L * (2 * kp * w.d + 2 * kp * (w.d + 1))
+    exps = q_heads * w.L * kp
+    hbm = w.units * 2 * (2 * w.d + 2 * w.d * w.Hkv / w.H) + 2 * kp * w.L * 4
+    clk = peaks["sm_max_mhz"] * 1e6
+    t = {"fma": flops / (2 * FFMA_PER_SM_CLK * NUM_SMS * clk) * 1e6, "mufu": exps / (MUFU_PER_SM_CLK * NUM_SMS * clk) * 1e6,
+         "hbm": hbm / (peaks["hbm_gbs"] * 1e9) * 1e6}
+    bound = max(t, key=t.get)
+    return {"workload": w.name + "_linformer_k256", "dtype": "bf16", "kp": kp, "steps": steps, "ms_per_step": ms,
+            "value": whole_job_rate(w.units, 1, ms), "unit": UNIT,
+            "roofline_path": {"t_fma_us": t["fma"], "t_mufu_us": t["mufu"], "t_hbm_us": t["hbm"], "bound": bound,
+                              "frac": t[bound] / (ms * 1e3)},
+            "input_sets": len(sets)}
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -600,6 +650,7 @@ def main():
         line["per_workload"] = entries
         line["decode"] = decode_entry(fv, dev, peaks)
         line["relu"] = relu_entry(fv, dev, peaks)
+        line["linformer"] = linformer_entry(fv, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r, heads, dt, threads = oracle_rate(w, 10.0)
         line["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": host_cores(), "blas_threads": threads,

@@ -169,6 +169,29 @@ FAVOR_API int favor_attention_relu(int dtype, const void* Q, const void* K, cons
                          void* out, int B, int H, int Hkv, int L, int d, int m, favor_stream_t stream);
 
 /*
+ * favor_linformer — Linformer projected attention (a second workload on the
+ * same machinery).
+ *
+ * Linformer notes page, section "4 Model": keys and values are projected along
+ * the sequence by E and F (k x L), and attention runs over the k projected
+ * rows: out = softmax(Q (E K)^T / sqrt(d)) (F V), per head.  One E and one F
+ * serve every head (the shared-projection option); query head h uses kv head
+ * h / (H / Hkv)'s projected rows.  E, F: device fp32 [kp, L] row-major (the
+ * caller's; random N(0, 1/L) entries stand in for trained ones).  dtype FAVOR_BF16 or
+ * FAVOR_F32 for Q, K, V and out; their layouts and the shape limits are those
+ * of favor_attention with m = kp (a multiple of 16 in [16, 512]) and, in
+ * addition, 2 * B * H <= 65535.  It runs on the CUDA cores in fp32: a
+ * projection kernel that sums each chunk of tokens into partial products, the
+ * fixed-order reduction, and the query pass with the exponential map over the
+ * kp projected keys (the softmax: a per-row maximum, exp, the weighted sum of
+ * F V and the division by the sum of the weights).  Scratch is allocated and
+ * freed stream-ordered on `stream`; errors as favor_attention.
+ */
+FAVOR_API int favor_linformer(int dtype, const void* Q, const void* K, const void* V, const float* E,
+                    const float* F, void* out, int B, int H, int Hkv, int L, int d, int kp,
+                    favor_stream_t stream);
+
+/*
  * favor_attention_host — end-to-end call on HOST buffers.
  *
  * Q, K, V, out are host pointers (pinned memory gives asynchronous copies;

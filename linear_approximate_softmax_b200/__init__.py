@@ -30,7 +30,7 @@ EXPORTS = [
     "favor_attention_f32", "favor_attention_host", "favor_partials_bytes", "favor_state_bytes",
     "favor_key_pass", "favor_state_reduce", "favor_query_pass", "favor_attention_noalloc", "favor_device_check",
     "favor_set_launch_overlap", "favor_decode_state_bytes", "favor_decode_init", "favor_decode_step",
-    "favor_attention_relu",
+    "favor_attention_relu", "favor_linformer",
 ]
 
 if not os.path.exists(LIB_PATH):
@@ -52,6 +52,8 @@ lib.favor_attention_host.argtypes = [_i] + _ATT
 lib.favor_attention_host.restype = _i
 lib.favor_attention_relu.argtypes = [_i] + _ATT
 lib.favor_attention_relu.restype = _i
+lib.favor_linformer.argtypes = [_i, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
+lib.favor_linformer.restype = _i
 lib.favor_partials_bytes.argtypes = [_i, _i, _i, _i, _i]
 lib.favor_partials_bytes.restype = _sz
 lib.favor_state_bytes.argtypes = [_i, _i, _i, _i]
@@ -166,6 +168,24 @@ def favor_attention_relu(Q, K, V, W, out=None, stream=None):
         out = torch.empty_like(Q)
     _check(lib.favor_attention_relu(code, _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(W, "W"), _dev(out, "out"),
                                     B, H, Hkv, L, d, m, _stream(stream)), "favor_attention_relu")
+    return out
+
+
+def favor_linformer(Q, K, V, E, F, out=None, stream=None):
+    """Linformer projected attention on device tensors: E, F are float32 [kp, L] projections."""
+    code = _dtype_code(Q)
+    if K.dtype != Q.dtype or V.dtype != Q.dtype or E.dtype != torch.float32 or F.dtype != torch.float32:
+        raise TypeError("Q, K, V must share a dtype and E, F must be float32")
+    if Q.dim() != 4 or K.dim() != 4 or V.shape != K.shape or E.dim() != 2 or E.shape != F.shape:
+        raise ValueError("expected Q [B,H,L,d], K and V [B,Hkv,L,d], E and F [kp,L]")
+    B, H, L, d = Q.shape
+    Hkv, kp = K.shape[1], E.shape[0]
+    if K.shape[0] != B or K.shape[2] != L or K.shape[3] != d or E.shape[1] != L:
+        raise ValueError("Q, K, V, E, F disagree on B, L or d")
+    if out is None:
+        out = torch.empty_like(Q)
+    _check(lib.favor_linformer(code, _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(E, "E"), _dev(F, "F"),
+                               _dev(out, "out"), B, H, Hkv, L, d, kp, _stream(stream)), "favor_linformer")
     return out
 
 

@@ -244,6 +244,29 @@ int relu_attention_impl(int dtype, const void* Q, const void* K, const void* V, 
   return FAVOR_OK;
 }
 
+// Linformer projected attention: projection kernel -> reduction -> projected query pass.
+int linformer_impl(int dtype, const void* Q, const void* K, const void* V, const float* E, const float* F,
+                   void* out, int B, int H, int Hkv, int L, int d, int kp, cudaStream_t st) {
+  FAVOR_TRY(check_dtype(dtype));
+  FAVOR_TRY(check_ptrs("favor_linformer", {Q, K, V, E, F, out}));
+  if (2L * B * H > 65535) return set_error(FAVOR_ERR_UNSUPPORTED, "favor_linformer: 2 * B * H must be at most 65535");
+  Plan pq, pk;
+  FAVOR_TRY(make_plan(B, H, Hkv, L, d, kp, &pq));
+  FAVOR_TRY(make_plan(2 * B, H, Hkv, L, d, kp, &pk));  // the projected keys ride as B more batches
+  keep_pool_mapped();
+  void* ws = nullptr;
+  const size_t st_off = round_up(pk.part_bytes, 256);
+  FAVOR_CUDA_TRY(cudaMallocAsync(&ws, st_off + pk.st_bytes, st), "favor_linformer scratch allocation");
+  char* base = static_cast<char*>(ws);
+  int rc = simt_linformer_proj(dtype, K, V, E, F, base, pk, B * Hkv, st);
+  if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, pk, st, false);
+  if (rc == FAVOR_OK) rc = simt_linformer_query(dtype, Q, base + st_off, out, pq, pk, st);
+  cudaError_t fe = cudaFreeAsync(ws, st);
+  if (rc != FAVOR_OK) return rc;
+  FAVOR_CUDA_TRY(fe, "favor_linformer scratch release");
+  return FAVOR_OK;
+}
+
 }  // namespace
 }  // namespace favor
 
@@ -276,6 +299,11 @@ int favor_attention_f32(const float* Q, const float* K, const float* V, const fl
 int favor_attention_relu(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,
                          int H, int Hkv, int L, int d, int m, favor_stream_t stream) {
   return relu_attention_impl(dtype, Q, K, V, W, out, B, H, Hkv, L, d, m, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int favor_linformer(int dtype, const void* Q, const void* K, const void* V, const float* E, const float* F, void* out,
+                    int B, int H, int Hkv, int L, int d, int kp, favor_stream_t stream) {
+  return linformer_impl(dtype, Q, K, V, E, F, out, B, H, Hkv, L, d, kp, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int favor_attention_host(int dtype, const void* Q, const void* K, const void* V, const float* W, void* out, int B,

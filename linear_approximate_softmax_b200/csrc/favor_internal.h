@@ -78,6 +78,13 @@ int simt_key_pass_relu(int dtype, const void* K, const void* V, const float* W, 
                        void* stream);
 int simt_query_pass_relu(int dtype, const void* Q, const float* W, const void* state, void* out, const Plan& p,
                          void* stream);
+// Linformer projected attention on the same machinery: the projections E K, F V of each kv
+// head written as key-pass partials of 2 * heads heads (plan pk: 2B batches), reduced by
+// simt_state_reduce, then the query pass with the exp map over the k projected keys (plan pq).
+int simt_linformer_proj(int dtype, const void* K, const void* V, const float* E, const float* F, void* partials,
+                        const Plan& pk, int heads, void* stream);
+int simt_linformer_query(int dtype, const void* Q, const void* state, void* out, const Plan& pq, const Plan& pk,
+                         void* stream);
 
 // ---- tensor-core kernels (sm_100a, bf16 storage) ------------------------------
 bool sm100_key_supported(const Plan& p);

@@ -286,10 +286,11 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
 }
 
 // grid (ceil(L/32), B*H), 256 threads.
+// W row f of kv head g at W + g * w_head + f * w_row (w_head = 0, w_row = D: one W for all heads).
 template <typename T, int D, int FMAP>
 __global__ void __launch_bounds__(kThreads) query_pass_kernel(
     const T* __restrict__ Q, const float* __restrict__ W, const float* __restrict__ S,
-    T* __restrict__ out, int L, int m, int H, int Hkv, float wscale) {
+    T* __restrict__ out, int L, int m, int H, int Hkv, float wscale, long w_head, int w_row) {
   constexpr int D1 = D + 1;
   constexpr int NE = (kQT * D1 + kThreads - 1) / kThreads;
   extern __shared__ float smem[];
@@ -305,6 +306,7 @@ __global__ void __launch_bounds__(kThreads) query_pass_kernel(
   const int q0 = blockIdx.x * kQT, qw = min(kQT, L - q0);
   const T* Qh = Q + static_cast<size_t>(bh) * L * D;
   const float* Sh = S + static_cast<size_t>(kvh) * m * D1;
+  const float* Wh = W + kvh * w_head;
 
   for (int i = tid; i < kQT * D; i += kThreads) {
     const int r = i / D, j = i % D;
@@ -315,7 +317,7 @@ __global__ void __launch_bounds__(kThreads) query_pass_kernel(
     __syncthreads();  // Qs ready / previous block done with Ws
     for (int i = tid; i < kFB * D; i += kThreads) {
       const int f = i / D, j = i % D;
-      Ws[f * D1 + j] = f < fbw ? W[static_cast<size_t>(f0 + f) * D + j] * wscale : 0.f;
+      Ws[f * D1 + j] = f < fbw ? Wh[static_cast<size_t>(f0 + f) * w_row + j] * wscale : 0.f;
     }
     __syncthreads();
     for (int i = tid; i < kQT * kFB; i += kThreads) {
@@ -368,6 +370,133 @@ __global__ void __launch_bounds__(kThreads) query_pass_kernel(
   }
 }
 
+// Linformer notes page, "4 Model": the projections E K and F V (k x d per kv head) of the keys
+// and values along the sequence.  grid (P, B*Hkv, ceil(k/64)), 256 threads: the CTA sums its
+// chunk of tokens for 64 projected rows into the key pass's partial-state layout, F V (with the
+// constant column 1 on chunk 0 only, so that the reduction's sum is 1) as head h and
+// kscale E K as head heads + h, every stabiliser 0.  Thread (ty, tx) owns rows 4 ty .. 4 ty + 3
+// and columns tx, tx + 16, ... of both products.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) linformer_proj_kernel(
+    const T* __restrict__ K, const T* __restrict__ V, const float* __restrict__ E, const float* __restrict__ F,
+    float* __restrict__ part_S, float* __restrict__ part_c, int L, int kp, int P, int chunk, int nsb, int heads,
+    float kscale) {
+  constexpr int D1 = D + 1;
+  constexpr int CT = D / 16;
+  constexpr int TT = 32;
+  extern __shared__ float smem[];
+  float* Es = smem;             // [64][TT + 1]
+  float* Fs = Es + 64 * (TT + 1);  // [64][TT + 1]
+  float* Ks = Fs + 64 * (TT + 1);  // [TT][D1]
+  float* Vs = Ks + TT * D1;        // [TT][D1]
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int p = blockIdx.x, head = blockIdx.y, j0 = blockIdx.z * 64;
+  const int t_begin = p * chunk, t_end = min(L, t_begin + chunk);
+  const T* Kh = K + static_cast<size_t>(head) * L * D;
+  const T* Vh = V + static_cast<size_t>(head) * L * D;
+  float ak[4][CT], av[4][CT];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < CT; ++c) ak[i][c] = av[i][c] = 0.f;
+  for (int t0 = t_begin; t0 < t_end; t0 += TT) {
+    const int tw = min(TT, t_end - t0);
+    __syncthreads();  // the previous step is done with the tiles
+    for (int i = tid; i < 64 * TT; i += kThreads) {
+      const int j = i / TT, t = i % TT;
+      const bool ok = j0 + j < kp && t < tw;
+      Es[j * (TT + 1) + t] = ok ? E[static_cast<size_t>(j0 + j) * L + t0 + t] : 0.f;
+      Fs[j * (TT + 1) + t] = ok ? F[static_cast<size_t>(j0 + j) * L + t0 + t] : 0.f;
+    }
+    for (int i = tid; i < TT * D; i += kThreads) {
+      const int t = i / D, c = i % D;
+      Ks[t * D1 + c] = t < tw ? to_f32(Kh[static_cast<size_t>(t0 + t) * D + c]) : 0.f;
+      Vs[t * D1 + c] = t < tw ? to_f32(Vh[static_cast<size_t>(t0 + t) * D + c]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int t = 0; t < TT; ++t) {
+      float e[4], f[4], kv[CT], vv[CT];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        e[i] = Es[(4 * ty + i) * (TT + 1) + t];
+        f[i] = Fs[(4 * ty + i) * (TT + 1) + t];
+      }
+#pragma unroll
+      for (int c = 0; c < CT; ++c) {
+        kv[c] = Ks[t * D1 + tx + 16 * c];
+        vv[c] = Vs[t * D1 + tx + 16 * c];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < CT; ++c) {
+          ak[i][c] = fmaf(e[i], kv[c], ak[i][c]);
+          av[i][c] = fmaf(f[i], vv[c], av[i][c]);
+        }
+    }
+  }
+  float* outV = part_S + (static_cast<size_t>(head) * P + p) * static_cast<size_t>(kp) * D1;
+  float* outK = part_S + (static_cast<size_t>(heads + head) * P + p) * static_cast<size_t>(kp) * D1;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = j0 + 4 * ty + i;
+    if (j >= kp) continue;
+#pragma unroll
+    for (int c = 0; c < CT; ++c) {
+      outK[static_cast<size_t>(j) * D1 + tx + 16 * c] = ak[i][c] * kscale;
+      outV[static_cast<size_t>(j) * D1 + tx + 16 * c] = av[i][c];
+    }
+    if (tx == 0) {
+      outK[static_cast<size_t>(j) * D1 + D] = 0.f;
+      outV[static_cast<size_t>(j) * D1 + D] = p == 0 ? 1.f : 0.f;
+      part_c[(static_cast<size_t>(head) * P + p) * nsb + j] = 0.f;
+      part_c[(static_cast<size_t>(heads + head) * P + p) * nsb + j] = 0.f;
+    }
+  }
+}
+
+template <typename T, int D>
+int launch_linformer_proj(const void* K, const void* V, const float* E, const float* F, void* partials,
+                          const Plan& pk, int heads, cudaStream_t st) {
+  constexpr int D1 = D + 1;
+  const size_t smem = sizeof(float) * (2 * 64 * 33 + 2 * 32 * D1);
+  auto kern = linformer_proj_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "projection attribute: %s", cudaGetErrorString(e));
+  dim3 grid(pk.P, heads, (pk.m + 63) / 64);
+  char* base = static_cast<char*>(partials);
+  const float kscale = static_cast<float>(std::pow(static_cast<double>(D), -0.25));
+  kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(K), static_cast<const T*>(V), E, F,
+                                     reinterpret_cast<float*>(base + pk.part_S_off),
+                                     reinterpret_cast<float*>(base + pk.part_c_off), pk.L, pk.m, pk.P, pk.chunk,
+                                     pk.nsb, heads, kscale);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "projection launch: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
+// softmax(Q Kp^T / sqrt(d)) Vp with the state S (head h: [F V | 1], head heads + h: d^-1/4 E K):
+// the query pass with the exp map, reading kv head h's projected keys as its W (row stride d + 1).
+template <typename T, int D>
+int launch_linformer_query(const void* Q, const void* state, void* out, const Plan& pq, const Plan& pk,
+                           cudaStream_t st) {
+  constexpr int D1 = D + 1;
+  const size_t smem = sizeof(float) * (kQT * D1 + kFB * D1 + kQT * (D1 + 1) + kQT * (pq.m + 1));
+  auto kern = query_pass_kernel<T, D, kExp>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "projected query attribute: %s", cudaGetErrorString(e));
+  dim3 grid((pq.L + kQT - 1) / kQT, pq.B * pq.H);
+  const float* S = reinterpret_cast<const float*>(static_cast<const char*>(state) + pk.st_S_off);
+  const int heads = pq.B * pq.Hkv;
+  const float* Wk = S + static_cast<size_t>(heads) * pq.m * D1;
+  kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(Q), Wk, S, static_cast<T*>(out), pq.L, pq.m, pq.H, pq.Hkv,
+                                     pq.wscale, static_cast<long>(pq.m) * D1, D1);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "projected query launch: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
 // d^-1/4: the input scaling of the ReLU map (no log2(e): no exponential)
 float relu_wscale(int d) { return static_cast<float>(std::pow(static_cast<double>(d), -0.25)); }
 
@@ -404,7 +533,7 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   const char* base = static_cast<const char*>(state);
   kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(Q), W,
                                      reinterpret_cast<const float*>(base + p.st_S_off),
-                                     static_cast<T*>(out), p.L, p.m, p.H, p.Hkv, wscale);
+                                     static_cast<T*>(out), p.L, p.m, p.H, p.Hkv, wscale, 0L, D);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "query pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
@@ -454,6 +583,26 @@ int simt_query_pass_relu(int dtype, const void* Q, const float* W, const void* s
                      : launch_query<float, 128, kRelu>(Q, W, state, out, p, st);
   return p.d == 64 ? launch_query<__nv_bfloat16, 64, kRelu>(Q, W, state, out, p, st)
                    : launch_query<__nv_bfloat16, 128, kRelu>(Q, W, state, out, p, st);
+}
+
+int simt_linformer_proj(int dtype, const void* K, const void* V, const float* E, const float* F, void* partials,
+                        const Plan& pk, int heads, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FAVOR_F32)
+    return pk.d == 64 ? launch_linformer_proj<float, 64>(K, V, E, F, partials, pk, heads, st)
+                      : launch_linformer_proj<float, 128>(K, V, E, F, partials, pk, heads, st);
+  return pk.d == 64 ? launch_linformer_proj<__nv_bfloat16, 64>(K, V, E, F, partials, pk, heads, st)
+                    : launch_linformer_proj<__nv_bfloat16, 128>(K, V, E, F, partials, pk, heads, st);
+}
+
+int simt_linformer_query(int dtype, const void* Q, const void* state, void* out, const Plan& pq, const Plan& pk,
+                         void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FAVOR_F32)
+    return pq.d == 64 ? launch_linformer_query<float, 64>(Q, state, out, pq, pk, st)
+                      : launch_linformer_query<float, 128>(Q, state, out, pq, pk, st);
+  return pq.d == 64 ? launch_linformer_query<__nv_bfloat16, 64>(Q, state, out, pq, pk, st)
+                    : launch_linformer_query<__nv_bfloat16, 128>(Q, state, out, pq, pk, st);
 }
 
 int simt_query_pass(int dtype, const void* Q, const float* W, const void* state, void* out,

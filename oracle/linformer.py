@@ -8,8 +8,10 @@ What it computes follows the Linformer notes page, section "4 Model": the keys
 and values of each head are projected along the sequence by two matrices E and
 F of k rows and n (here L) columns, and attention runs over the k projected
 rows:  out = softmax(Q (E K)^T / sqrt(d)) (F V).  The pages use trained E and
-F; the tests pass seeded Gaussian ones with entries N(0, 1/k), the plainest
-stand-in (a random projection of the sequence).  One E and one F serve every
+F; the tests pass seeded Gaussian ones with entries N(0, 1/L), the plainest
+stand-in: a random projection of the sequence whose rows, like an average over
+the tokens, keep the scale of the rows of K and V (so outputs stay on V's scale
+and the tolerances of the other workloads apply as stated).  One E and one F serve every
 head of a call (the page's shared-projection option); query heads that share a
 key/value head (multi-query layout) share its projected rows.
 """
@@ -19,9 +21,9 @@ import numpy as np
 
 
 def projection(seed, k, L):
-    """A seeded k x L matrix with N(0, 1/k) entries (numpy's generator; an input, not part of the method)."""
+    """A seeded k x L matrix with N(0, 1/L) entries (numpy's generator; an input, not part of the method)."""
     rng = np.random.default_rng(seed)
-    return rng.standard_normal((k, L)) / math.sqrt(k)
+    return rng.standard_normal((k, L)) / math.sqrt(L)
 
 
 def linformer_attention(Q, K, V, E, F):

@@ -57,7 +57,7 @@ def test_linear_in_the_values_and_inside_the_projected_hull():
     assert np.all(a >= Vp.min(axis=2, keepdims=True) - 1e-12) and np.all(a <= Vp.max(axis=2, keepdims=True) + 1e-12)
 
 
-def test_projection_entries_have_variance_one_over_k():
+def test_projection_entries_have_variance_one_over_L():
     E = linformer.projection(41, 64, 4096)
-    assert abs(E.mean()) < 4 / math.sqrt(E.size) / math.sqrt(64)
-    assert abs(E.var() * 64 - 1.0) < 0.02
+    assert abs(E.mean()) < 4 / math.sqrt(E.size) / math.sqrt(4096)
+    assert abs(E.var() * 4096 - 1.0) < 0.02
