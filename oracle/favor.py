@@ -238,6 +238,43 @@ def decode_outputs(Q, K, V, W):
 
 
 # --------------------------------------------------------------------------
+# Trigonometric random features, the comparison point of the feature-map
+# study ("Rethinking Attention with Performers", 제안 방법 / proposed method:
+# positive features instead of the usual sin/cos ones; 주요 결과 / main results:
+# positive and orthogonal features lower the error).  With r rows of W,
+# phi(x') = exp(|x'|^2/2) / sqrt(r) [sin(W x'), cos(W x')] (2r features):
+# sin a sin b + cos a cos b = cos(a - b) and E_w cos(w.z) = exp(-|z|^2/2) for
+# w ~ N(0, I), so E[phi(q')^T phi(k')] = exp(q'.k').  Its weights can be
+# negative, so no stabiliser applies and the ratio can leave V's hull.
+# --------------------------------------------------------------------------
+def trig_features(X, W):
+    """exp(|x'|^2/2) / sqrt(r) [sin(W x'), cos(W x')] for every scaled row x' of X ([n, 2r])."""
+    W = np.asarray(W, dtype=np.float64)
+    Xs = scale_inputs(X)
+    u = Xs @ W.T
+    amp = np.exp(0.5 * np.sum(Xs * Xs, axis=1, keepdims=True)) / math.sqrt(W.shape[0])
+    return amp * np.concatenate([np.sin(u), np.cos(u)], axis=1)
+
+
+def trig_attention(Q, K, V, W):
+    """The linear-time estimate with trigonometric features, per kv head, fp64 (shapes as favor_attention)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, L, d = Q.shape
+    G = H // K.shape[1]
+    out = np.empty((B, H, L, d), dtype=np.float64)
+    for b in range(B):
+        for g in range(K.shape[1]):
+            V1 = np.concatenate([V[b, g], np.ones((V.shape[2], 1))], axis=1)
+            S = trig_features(K[b, g], W).T @ V1
+            for h in range(g * G, (g + 1) * G):
+                nz = trig_features(Q[b, h], W) @ S
+                out[b, h] = nz[:, :d] / nz[:, d:d + 1]
+    return out
+
+
+# --------------------------------------------------------------------------
 # Generalised kernelizable attention, f = ReLU ("Rethinking Attention with
 # Performers", Abstract: the method also approximates kernelizable attention
 # other than softmax; 연구 질문 / research questions, RQ5).  The pages name no

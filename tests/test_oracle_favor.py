@@ -232,3 +232,41 @@ def test_relu_attention_with_identical_keys_returns_the_mean_value():
     W = favor.make_features(29, 32, 16)
     out = favor.relu_attention(Q, K, V, W)
     np.testing.assert_allclose(out[0, 0], np.broadcast_to(V[0, 0].mean(axis=0), (20, 16)), rtol=1e-11, atol=1e-12)
+
+
+# ---- trigonometric random features (the study's comparison point) ---------------------
+def test_trig_feature_product_is_unbiased_for_softmax_kernel():
+    d = 16
+    rng = np.random.default_rng(42)
+    q = rng.standard_normal(d) * 0.45
+    k = rng.standard_normal(d) * 0.45
+    est = np.empty(2000)
+    for s in range(est.size):
+        W = favor.make_features(20_000 + s, d, d, orthogonal=False)
+        est[s] = float(favor.trig_features(q[None], W)[0] @ favor.trig_features(k[None], W)[0])
+    target = math.exp(float(q @ k) / math.sqrt(d))
+    se = est.std(ddof=1) / math.sqrt(est.size)
+    assert abs(est.mean() - target) < 3.5 * se, (est.mean(), target, se)
+    assert se < 0.05 * target
+
+
+def test_trig_linear_order_equals_quadratic_form():
+    Q, K, V = _inputs(1, 2, 1, 30, 16, scale=0.6, seed=43)
+    W = favor.make_features(44, 24, 16)
+    want = np.empty_like(Q)
+    for h in range(2):
+        A = favor.trig_features(Q[0, h], W) @ favor.trig_features(K[0, 0], W).T
+        want[0, h] = (A @ V[0, 0]) / A.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(favor.trig_attention(Q, K, V, W), want, rtol=1e-9, atol=1e-10)
+
+
+def test_trig_features_reproduce_the_gaussian_kernel_identity():
+    # for one frequency row w: phi(x)^T phi(y) r = exp(|x'|^2/2 + |y'|^2/2) cos(w.(x' - y')), by the
+    # angle-difference identity, whatever w is
+    rng = np.random.default_rng(45)
+    x, y = rng.standard_normal(8), rng.standard_normal(8)
+    W = rng.standard_normal((1, 8))
+    xs, ys = x * 8 ** -0.25, y * 8 ** -0.25
+    want = math.exp(0.5 * (xs @ xs + ys @ ys)) * math.cos(float(W[0] @ (xs - ys)))
+    got = float(favor.trig_features(x[None], W)[0] @ favor.trig_features(y[None], W)[0])
+    assert abs(got - want) < 1e-12 * abs(want) + 1e-15
