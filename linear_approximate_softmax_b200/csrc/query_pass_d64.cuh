@@ -22,8 +22,8 @@
 // Each epilogue warpgroup owns, in tensor memory, its Q operand, two U buffers and its O
 // accumulator.  Blocks of 64 features alternate between the two U buffers; the epilogue reads a
 // block's U into registers and writes phi' over the same columns, so the epilogue never waits
-// for a contraction: the next block's U is already in the other buffer, and a buffer is reused
-// (two blocks later) only once the contraction that read it has completed.  The Q conversion
+// for a contraction: the next block's U is already in the other buffer, and a buffer is
+// re-projected (two blocks later) right after the contraction that reads it is issued.  The Q conversion
 // and the output run in their own warpgroup, off the exponential loop.
 //
 // Stabiliser: c_q is the exact maximum of the row's first block (two passes over it); later
@@ -200,9 +200,10 @@ __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
       }
     } else if (warp == 1 || warp == 2) {
       // ---------------- MMA issuer of epilogue warpgroup w: its tiles w, w + 2, ... ----------------
-      // Two streams over the warpgroup's blocks a = tile * nb + j: MMA1(a) into U buffer a % 2,
-      // once the buffer's previous contraction (block a - 2) has completed and, for a tile's first
-      // block, once its Q operand is converted; MMA2(a) once the epilogue has written phi'(a).
+      // Two streams over the warpgroup's blocks a = tile * nb + j: MMA2(a) once the epilogue has
+      // written phi'(a), then at once MMA1(a + 2) into the same U buffer (for a tile's first block,
+      // once its Q operand is converted): the tensor core runs one thread's MMAs in issue order, so
+      // the projection cannot overwrite phi'(a) before the contraction has read it.
       if (lane == 0) {
         const int w = warp - 1;
         const uint32_t tw = tbase + w * C::T_WG;
@@ -214,7 +215,8 @@ __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
         int a1 = 0, t1 = 0, j1 = 0;  // next projection: block a1 = t1 * nb + j1
         auto issue_mma1 = [&]() -> bool {
           if (j1 == 0 && !mbar_wait(bar(C::B_CVT + 2 * w + (t1 & 1)), (t1 >> 1) & 1, abort_flag, err)) return false;
-          if (a1 >= 2 && !mbar_wait(bar(C::B_M2 + 2 * w + (a1 & 1)), ((a1 - 2) >> 1) & 1, abort_flag, err)) return false;
+          // No wait for MMA2(a1 - 2), which reads phi' from the same columns: this thread issued it
+          // just before, and the tensor core executes one thread's MMAs in issue order.
           tc_fence_after();
           const uint32_t d = dU + (a1 & 1) * C::FB;
 #pragma unroll
