@@ -76,7 +76,12 @@ def load_peaks():
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a kernel on a workload,
 # from one ncu capture of the kernel as it stands; an entry is removed whenever its kernel changes
 # (the bench then reports traffic null until the kernel is captured again).
-PROFILED_TRAFFIC = {}
+PROFILED_TRAFFIC = {
+    # query_pass_d64_sm100 as of "issue the next projection right after the contraction ..."
+    ("bf16_L16384_heavykeys", "query_pass"): 157.59e6,
+    # key_pass_pp_sm100, unchanged since "Overlap consecutive kernels with programmatic dependent launch"
+    ("bf16_L16384_heavykeys", "key_pass"): 210.31e6,
+}
 
 # Per-SM issue rates of one B200 SM per clock, times 148 SMs and the maximum SM clock: the MUFU
 # ex2 rate (16 results per clock) bounds the exponentials; the fp32 FMA rate (128 per clock, 2
