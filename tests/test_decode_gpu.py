@@ -39,6 +39,9 @@ def run_decode(Q, K, V, W):
     (torch.bfloat16, 2, 4, 1, 1000, 128, 256),   # multi-query: four query heads share one kv head
     (torch.bfloat16, 1, 6, 2, 400, 64, 512),
     (torch.float32, 1, 2, 2, 300, 64, 128),
+    (torch.bfloat16, 1, 64, 1, 120, 128, 512),   # the most query heads per kv head, the most features
+    (torch.float32, 2, 17, 1, 150, 64, 16),      # an odd group of query heads, two features per CTA
+    (torch.bfloat16, 3, 10, 2, 100, 128, 208),   # 26 features per CTA: not a power of two
 ])
 def test_decode_matches_oracle(dtype, B, H, Hkv, T, d, m, parity_report):
     Q, K, V = wl.random_inputs(B, H, Hkv, T, d, dtype, seed=T + d)
