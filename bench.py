@@ -79,8 +79,8 @@ def load_peaks():
 PROFILED_TRAFFIC = {
     # query_pass_d64_sm100 as of "issue the next projection right after the contraction ..."
     ("bf16_L16384_heavykeys", "query_pass"): 157.59e6,
-    # key_pass_pp_sm100, unchanged since "Overlap consecutive kernels with programmatic dependent launch"
-    ("bf16_L16384_heavykeys", "key_pass"): 210.31e6,
+    # key_pass_pp_sm100 as of "256 features per key-pass CTA, key norms in their own warp ..."
+    ("bf16_L16384_heavykeys", "key_pass"): 205.87e6,
 }
 
 # Per-SM issue rates of one B200 SM per clock, times 148 SMs and the maximum SM clock: the MUFU

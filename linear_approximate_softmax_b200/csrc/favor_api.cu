@@ -95,9 +95,10 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
   const int heads = B * Hkv;
   const int tiles = (L + kTileTokens - 1) / kTileTokens;
   // Key chunks: the tensor-core key pass runs one CTA per SM for each (kv head,
-  // 128-feature group, chunk).  Pick the chunk count that minimises the
+  // feature group, chunk).  Pick the chunk count that minimises the
   // makespan in waves of CTAs, counting half a tile of start-up per wave.
-  const long units = static_cast<long>(heads) * ((m + 127) / 128);
+  const int nfeat = key_features_per_cta(d, m);
+  const long units = static_cast<long>(heads) * ((m + nfeat - 1) / nfeat);
   double best = 1e300;
   int best_ct = tiles;
   for (int P = 1; P <= tiles; ++P) {

@@ -88,6 +88,9 @@ int simt_linformer_query(int dtype, const void* Q, const void* state, void* out,
 
 // ---- tensor-core kernels (sm_100a, bf16 storage) ------------------------------
 bool sm100_key_supported(const Plan& p);
+// Features per CTA of the tensor-core key pass: 256 for d = 64 with m > 128 (each of its two
+// epilogue warpgroups takes 128 features of every key tile), else 128.
+inline int key_features_per_cta(int d, int m) { return d == 64 && m > 128 ? 256 : 128; }
 bool sm100_query_supported(const Plan& p);
 int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st,
                    bool overlap);

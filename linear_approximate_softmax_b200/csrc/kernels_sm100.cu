@@ -406,47 +406,56 @@ __global__ void __launch_bounds__(kThreads, 1) key_pass_sm100(
 }
 
 // ============================================================================
-// Key pass, d = 64: the two epilogue warpgroups take alternate tiles
+// Key pass, d = 64: two epilogue warpgroups, each with its own projection, weights and accumulator
 // ============================================================================
 // Each warpgroup owns a U^T buffer, a phi buffer and an S accumulator in tensor
 // memory, its own running stabilisers and its own MMA-issuing thread (warp 1 for
 // warpgroup 0, warp 2 for warpgroup 1).  The epilogue releases U^T as soon as it
 // has read it, so the next tile's projection runs while this tile's exponentials
-// and its contraction finish; phi goes to its own buffer.  A warpgroup prepares
-// (norms, fp16 conversion) the tile after its current one before waiting for the
-// current U^T.  The normaliser column sum_t phi is accumulated by the epilogue
-// itself, in fp32.  At the end the two accumulators are merged exactly:
-// S = 2^(c0-c) S0 + 2^(c1-c) S1.
+// and its contraction finish; phi goes to its own buffer.  Warp 3 computes every
+// tile's key norms as soon as the tile lands, once for both warpgroups.  The
+// normaliser column sum_t phi is accumulated by the epilogue itself, in fp32.
+//  * WIDE (m > 128): a CTA covers 256 features; warpgroup w takes features 128 w ..
+//    128 w + 127 of every tile, so each K/V tile and its norms serve 256 features and
+//    the grid is half as large.
+//  * otherwise: a CTA covers 128 features; the warpgroups take alternate tiles, and at
+//    the end the two accumulators are merged exactly: S = 2^(c0-c) S0 + 2^(c1-c) S1.
+template <bool WIDE>
 struct KeyPP {
   static constexpr int D = 64;
-  // warp 0 TMA producer, warps 1-2 MMA issuers, warp 3 idle, warps 4-11 two epilogue
+  static constexpr int NFEAT = WIDE ? 256 : 128;  // features per CTA
+  // warp 0 TMA producer, warps 1-2 MMA issuers, warp 3 key norms, warps 4-11 two epilogue
   // warpgroups (each covers the four TMEM lane quarters once, as warp % 4)
   static constexpr int THREADS = 384;
   static constexpr int EPI0 = 4;
-  static constexpr int NST = 5;  // K/V stages: a tile's norms are taken two tiles ahead of its use
+  static constexpr int NST = WIDE ? 4 : 5;  // K/V stages (the wide W' takes the fifth's room)
   static constexpr int TILE = 128 * 64 * 2;
   // TMEM columns: warpgroup w owns U^T at 256 w, phi at 256 w + 128 (bf16 pairs), S at 256 w + 192
   static constexpr int T_U = 0, T_P = 128, T_S = 192, T_STRIDE = 256;
-  // W' = hi + lo in bf16, each 128 features x 64 dims, K-major SW128 (the A operands of MMA1)
-  static constexpr int S_WHI = 0, S_WLO = 128 * 128;
-  static constexpr int S_K = S_WLO + 128 * 128;
+  // W' = hi + lo in bf16, each NFEAT features x 64 dims, K-major SW128 (the A operands of MMA1;
+  // warpgroup w of a wide CTA starts at row 128 w)
+  static constexpr int S_WHI = 0, S_WLO = NFEAT * 128;
+  static constexpr int S_K = S_WLO + NFEAT * 128;
   static constexpr int S_V = S_K + NST * TILE;
   static constexpr int S_NRM = S_V + NST * TILE;    // per stage: -n(k) [128]
   static constexpr int S_CW = S_NRM + NST * 512;    // final stabilisers and normalisers, [2][2][128]
   static constexpr int S_BAR = S_CW + 2048;
-  static constexpr int B_KVF = 0, B_KVE = NST, B_NRM = 2 * NST, B_D1F = B_NRM + 2, B_UE = B_D1F + 2,
-                       B_PHI = B_UE + 2, B_SDONE = B_PHI + 2, NBAR = B_SDONE + 2;
+  // PHI and SDONE come in halves per warpgroup (2 w + h): the weights of tokens 64 h .. 64 h + 63
+  // and the contraction steps that read them
+  static constexpr int B_KVF = 0, B_KVE = NST, B_NRM = 2 * NST, B_D1F = B_NRM + NST, B_UE = B_D1F + 2,
+                       B_PHI = B_UE + 2, B_SDONE = B_PHI + 4, NBAR = B_SDONE + 4;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int SMEM = S_ABORT + 16 + 1024;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-__global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
+template <bool WIDE>
+__global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const float* __restrict__ W,
     float* __restrict__ part_S, float* __restrict__ part_c, int L, int m, int P, int chunk, int nsb, float wscale,
     float nscale) {
-  using C = KeyPP;
+  using C = KeyPP<WIDE>;
   constexpr int D = C::D;
   extern __shared__ unsigned char smem_raw[];
   griddep_launch_dependents();  // the next kernel on the stream may be scheduled as SMs free up
@@ -456,9 +465,11 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grp = blockIdx.x, p = blockIdx.y, head = blockIdx.z;
-  const int f0 = grp * 128, gw = min(128, m - f0);
+  const int f0 = grp * C::NFEAT, gw = min(C::NFEAT, m - f0);
   const int t_begin = p * chunk, t_end = min(L, t_begin + chunk);
   const int ntiles = (t_end - t_begin + 127) / 128;
+  // tiles of warpgroup w: all of them (wide), or w, w + 2, ...
+  constexpr int TSTEP = WIDE ? 1 : 2;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
   uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
   float* nrm = reinterpret_cast<float*>(smem + C::S_NRM);
@@ -468,14 +479,16 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(bar(C::B_KVF + s), 1);
-      mbar_init(bar(C::B_KVE + s), 1);
+      mbar_init(bar(C::B_KVE + s), WIDE ? 2 : 1);  // the contraction(s) of the stage's tile
+      mbar_init(bar(C::B_NRM + s), 1);  // the norm warp, once per tile of the stage
     }
     for (int w = 0; w < 2; ++w) {
-      mbar_init(bar(C::B_NRM + w), 4);  // one arrival per epilogue warp
       mbar_init(bar(C::B_D1F + w), 1);
       mbar_init(bar(C::B_UE + w), 4);
-      mbar_init(bar(C::B_PHI + w), 4);
-      mbar_init(bar(C::B_SDONE + w), 1);
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(bar(C::B_PHI + 2 * w + h), 4);
+        mbar_init(bar(C::B_SDONE + 2 * w + h), 1);
+      }
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -495,7 +508,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
   // W' = hi + lo (bf16) as the K-major 128B-swizzled A operands of MMA1: row f, 16-byte chunk c
   // at c ^ (f % 8); the pair keeps ~16 bits of W', so the exponents stay within the bf16
   // output tolerance on heavy-tailed keys
-  for (int item = tid; item < 128 * 8; item += C::THREADS) {
+  for (int item = tid; item < C::NFEAT * 8; item += C::THREADS) {
     const int f = item >> 3, c = item & 7;
     uint32_t hi[4], lo[4];
 #pragma unroll
@@ -542,7 +555,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
         mbar_wait(bar(C::B_KVF + i % C::NST), (i / C::NST) & 1, abort_flag, err, 200000000ull);
     }
   } else if (warp == 1 || warp == 2) {
-    // ---------------- MMA issuer of warpgroup w: tiles w, w + 2, ... ----------------
+    // ---------------- MMA issuer of warpgroup w: its tiles (all, or w, w + 2, ...) ----------------
     // The next tile's projection is issued as soon as the epilogue has read this tile's
     // U^T, ahead of this tile's contraction.
     if (lane == 0) {
@@ -551,53 +564,96 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       const uint32_t idv = idesc_bf16(128, D, false, true);  // V tile as an MN-major B operand
       const uint32_t dU = tbase + w * C::T_STRIDE + C::T_U, dP = tbase + w * C::T_STRIDE + C::T_P,
                      dS = tbase + w * C::T_STRIDE + C::T_S;
+      const uint32_t wrow = WIDE ? w * 128 * 128 : 0;  // this warpgroup's rows of W'
       auto mma1 = [&](int i) {  // U^T = (W'hi + W'lo) K^T
         const int s = i % C::NST;
 #pragma unroll
         for (int ks = 0; ks < 2 * (D / 16); ++ks) {
           const int kk = ks % (D / 16);
-          mma_ss(dU, sdesc_sw128(sbase + (ks < D / 16 ? C::S_WHI : C::S_WLO) + 32 * kk, 16, 1024),
+          mma_ss(dU, sdesc_sw128(sbase + (ks < D / 16 ? C::S_WHI : C::S_WLO) + wrow + 32 * kk, 16, 1024),
                  sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * kk, 16, 1024), id1, ks > 0 ? 1u : 0u);
         }
         mma_commit(bar(C::B_D1F + w));
       };
       int cnt = 0;
-      bool ok = w < ntiles && mbar_wait(bar(C::B_KVF + w % C::NST), (w / C::NST) & 1, abort_flag, err);
+      const int first = WIDE ? 0 : w;
+      bool ok = first < ntiles && mbar_wait(bar(C::B_KVF + first % C::NST), (first / C::NST) & 1, abort_flag, err);
       if (ok) {
         tc_fence_after();
-        mma1(w);
+        mma1(first);
       }
-      for (int i = w; i < ntiles && ok; i += 2, ++cnt) {
+      for (int i = first; i < ntiles && ok; i += TSTEP, ++cnt) {
         const int s = i % C::NST;
-        if (i + 2 < ntiles) {
+        if (i + TSTEP < ntiles) {
           if (!mbar_wait(bar(C::B_UE + w), cnt & 1, abort_flag, err)) break;  // U^T of tile i read
-          const int s2 = (i + 2) % C::NST;
-          if (!mbar_wait(bar(C::B_KVF + s2), ((i + 2) / C::NST) & 1, abort_flag, err)) break;  // tile i + 2 landed
+          const int s2 = (i + TSTEP) % C::NST;
+          if (!mbar_wait(bar(C::B_KVF + s2), ((i + TSTEP) / C::NST) & 1, abort_flag, err)) break;  // the next tile landed
           tc_fence_after();
-          mma1(i + 2);
+          mma1(i + TSTEP);
         }
-        if (!mbar_wait(bar(C::B_PHI + w), cnt & 1, abort_flag, err)) break;
-        tc_fence_after();
+        // MMA2: S_w += phi^T V, 16 tokens per step, each half of the tile as soon as its weights are in
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!(ok = mbar_wait(bar(C::B_PHI + 2 * w + h), cnt & 1, abort_flag, err))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {  // MMA2: S_w += phi^T V, 16 tokens per step
-          const uint64_t bv = sdesc_sw128(sbase + C::S_V + s * C::TILE + 2048 * ks, 16, 1024);
-          mma_ts(dS, dP + 8 * ks, bv, idv, (cnt > 0 || ks > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            const int ks = 4 * h + k;
+            const uint64_t bv = sdesc_sw128(sbase + C::S_V + s * C::TILE + 2048 * ks, 16, 1024);
+            mma_ts(dS, dP + 8 * ks, bv, idv, (cnt > 0 || ks > 0) ? 1u : 0u);
+          }
+          if (h == 1) mma_commit(bar(C::B_KVE + s));
+          mma_commit(bar(C::B_SDONE + 2 * w + h));
         }
-        mma_commit(bar(C::B_KVE + s));
-        mma_commit(bar(C::B_SDONE + w));
       }
-      const int mine = (ntiles + 1 - w) / 2;
-      if (mine > 0) mbar_wait(bar(C::B_SDONE + w), (mine - 1) & 1, abort_flag, err, 200000000ull);
+      const int mine = WIDE ? ntiles : (ntiles + 1 - w) / 2;
+      if (mine > 0) mbar_wait(bar(C::B_SDONE + 2 * w + 1), (mine - 1) & 1, abort_flag, err, 200000000ull);
+    }
+  } else {
+    // ---------------- key norms: -n(k) = -|k|^2 nscale per token (-inf past the chunk end) ----------------
+    // Lane l takes tokens l, l + 32, l + 64, l + 96 of each tile, two at a time.  The 16-byte chunks of a swizzled
+    // row are summed in any order; token t starts at chunk t % 8, so the eight lanes of a
+    // shared-memory wavefront hit different banks.  The stage's norms are overwritten only after
+    // the tile that last used it has been contracted, which needs its exponentials, which need
+    // these norms, so no other wait is needed.
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % C::NST;
+      if (!mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err)) break;
+#pragma unroll 1
+      for (int r2 = 0; r2 < 2; ++r2) {  // two tokens at a time, for independent chains
+        const int ta = lane + 64 * r2, tb = ta + 32;
+        const uint4* ra = reinterpret_cast<const uint4*>(smem + C::S_K + s * C::TILE + ta * 128);
+        const uint4* rb = reinterpret_cast<const uint4*>(smem + C::S_K + s * C::TILE + tb * 128);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 va = ra[c ^ (ta & 7)], vb = rb[c ^ (tb & 7)];
+          const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 xa = make_float2(__uint_as_float(wa[q] << 16), __uint_as_float(wa[q] & 0xFFFF0000u));
+            const float2 xb = make_float2(__uint_as_float(wb[q] << 16), __uint_as_float(wb[q] & 0xFFFF0000u));
+            acc[q & 1] = __ffma2_rn(xa, xa, acc[q & 1]);
+            acc[2 + (q & 1)] = __ffma2_rn(xb, xb, acc[2 + (q & 1)]);
+          }
+        }
+        const float sa = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
+        const float sb = (acc[2].x + acc[2].y) + (acc[3].x + acc[3].y);
+        nrm[s * 128 + ta] = (t_begin + 128 * i + ta < t_end) ? -sa * nscale : -INFINITY;
+        nrm[s * 128 + tb] = (t_begin + 128 * i + tb < t_end) ? -sb * nscale : -INFINITY;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_NRM + s));  // release: the 128 norms are stored
     }
   }
   } else {
     setmaxnreg_inc<kRegsHigh>();
-    // ---------------- epilogue warpgroup ewg: tiles ewg, ewg + 2, ... ----------------
+    // ---------------- epilogue warpgroup ewg: its tiles (all, or ewg, ewg + 2, ...) ----------------
     const int eq = warp & 3;
     const int ewg = (warp - C::EPI0) >> 2;
-    const int frow = eq * 32 + lane;
-    const bool fvalid = frow < gw;
-    // Each thread owns feature f0 + frow and reads each U^T value of its row once.  Its
+    const int frow = eq * 32 + lane;                  // the thread's TMEM lane (row of U^T and S)
+    const int fr = (WIDE ? 128 * ewg : 0) + frow;     // its feature, counted from f0
+    const bool fvalid = fr < gw;
+    // Each thread owns feature f0 + fr and reads each U^T value of its row once.  Its
     // stabiliser c is that feature's running max exponent over the tiles seen so far,
     // raised (with an exact rescale of its S row and normaliser) only when a tile exceeds
     // it by more than 2^kTau, and never below floor = |w|^2 log2(e)/2 - 64: by completing
@@ -608,7 +664,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     {
       float w2 = 0.f;
       if (fvalid) {
-        const float4* wr = reinterpret_cast<const float4*>(W + static_cast<size_t>(f0 + frow) * D);
+        const float4* wr = reinterpret_cast<const float4*>(W + static_cast<size_t>(f0 + fr) * D);
 #pragma unroll
         for (int k = 0; k < D / 4; ++k) {
           const float4 v = wr[k];
@@ -620,41 +676,13 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     float c_run = floor_c, tmax = -INFINITY, zsum = 0.f;  // zsum: this feature's normaliser sum_t phi
     const uint32_t cU = ewg * C::T_STRIDE + C::T_U, cP = ewg * C::T_STRIDE + C::T_P,
                    cS = ewg * C::T_STRIDE + C::T_S;
-    // The key norms of tile i, one key row (token frow) per thread: -n(k) = -|k|^2 nscale
-    // (-inf past the chunk end), for the whole warpgroup once all four warps have arrived on
-    // B_NRM.  The 16-byte chunks of a swizzled row are summed in any order; thread frow starts
-    // at chunk frow % 8, so the eight threads of a shared-memory wavefront hit different banks.
-    auto prepare_tile = [&](int i) {
-      const int s = i % C::NST;
-      mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err);
-      const uint4* row = reinterpret_cast<const uint4*>(smem + C::S_K + s * C::TILE + frow * 128);
-      float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = row[c ^ (frow & 7)];
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 x = make_float2(__uint_as_float(wv[q] << 16), __uint_as_float(wv[q] & 0xFFFF0000u));
-          acc[q & 1] = __ffma2_rn(x, x, acc[q & 1]);
-        }
-      }
-      const float sum = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
-      nrm[s * 128 + frow] = (t_begin + 128 * i + frow < t_end) ? -sum * nscale : -INFINITY;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_NRM + ewg));  // this warp's 32 norms are stored
-    };
     int cnt = 0;
-    if (ewg < ntiles) prepare_tile(ewg);
-    for (int i = ewg; i < ntiles; i += 2, ++cnt) {
+    for (int i = WIDE ? 0 : ewg; i < ntiles; i += TSTEP, ++cnt) {
       const int s = i % C::NST;
       mbar_wait(bar(C::B_D1F + ewg), cnt & 1, abort_flag, err);
-      // every warp's norms of tile i are visible once all four have arrived for it (this
-      // warp waits before arriving for tile i + 2, so the phase cannot have moved on)
-      mbar_wait(bar(C::B_NRM + ewg), cnt & 1, abort_flag, err);
-      // the norms of tile i + 2, two tiles ahead (after U^T of i has arrived, so that each
-      // warp's arrival stays one phase ahead of the waits on it)
-      if (i + 2 < ntiles) prepare_tile(i + 2);
+      // the norms of tile i (the norm warp cannot have moved on to the stage's next tile: that
+      // tile is loaded only after this one has been contracted)
+      mbar_wait(bar(C::B_NRM + s), (i / C::NST) & 1, abort_flag, err);
       // this tile's U^T row into registers (one read), then release it to the next projection
       float ut[128];
 #pragma unroll
@@ -663,11 +691,14 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_UE + ewg));
-      if (cnt >= 1) mbar_wait(bar(C::B_SDONE + ewg), (cnt - 1) & 1, abort_flag, err);  // phi buffer free, S final
-      tc_fence_after();
-      // the previous tile raised the running max: rescale S and the normaliser now
+      // the previous tile raised the running max: rescale S and the normaliser now, once the
+      // previous tile's contraction is complete
       const bool need = tmax > c_run + kTau;
-      if (__any_sync(0xffffffffu, need)) scale_tmem_row(taddr(tbase, eq, cS), D / 8, need ? ex2(c_run - tmax) : 1.f);
+      if (__any_sync(0xffffffffu, need)) {
+        if (cnt >= 1) mbar_wait(bar(C::B_SDONE + 2 * ewg + 1), (cnt - 1) & 1, abort_flag, err);
+        tc_fence_after();
+        scale_tmem_row(taddr(tbase, eq, cS), D / 8, need ? ex2(c_run - tmax) : 1.f);
+      }
       if (need) {
         zsum *= ex2(c_run - tmax);
         c_run = tmax;
@@ -678,6 +709,11 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
       const float4* nv = reinterpret_cast<const float4*>(nrm + s * 128);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
+        if ((q4 & 1) == 0) {  // a new half: its phi columns are free once the previous tile's
+          const int h = q4 >> 1;  // contraction steps that read them are complete
+          if (cnt >= 1) mbar_wait(bar(C::B_SDONE + 2 * ewg + h), (cnt - 1) & 1, abort_flag, err);
+          tc_fence_after();
+        }
         uint32_t wph[16];
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {  // two tokens per packed fp32x2 operation
@@ -695,32 +731,49 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
         }
         // (a feature past m has W' = 0; its S row is computed but never written out)
         tmem_st16(taddr(tbase, eq, cP + 16 * q4), wph);  // phi, bf16 pairs
+        if (q4 & 1) {  // this half's weights are in: its contraction steps may go
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::B_PHI + 2 * ewg + (q4 >> 1)));
+        }
       }
       zsum += zs2.x + zs2.y;
       tmax = fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3]));
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::B_PHI + ewg));
     }
     if (!fvalid) zsum = 0.f;
-    // merge the two accumulators row by row and write this group's partial state, once the
-    // kernels before this one on the stream (which may read the partial state) have completed
+    // write this group's partial state (merging the two accumulators row by row when they took
+    // alternate tiles), once the kernels before this one on the stream (which may read the
+    // partial state) have completed.  The rows go through shared memory (the K/V stages are free
+    // once every MMA has completed) so that the partial state is written with coalesced 16-byte
+    // stores; a row stride of D + 1 floats (odd) keeps the 32 rows of a warp on different banks.
     griddep_wait();
+    float* stg = reinterpret_cast<float*>(smem + C::S_K);
+    if constexpr (WIDE) {
+      if (ntiles > 0) mbar_wait(bar(C::B_SDONE + 2 * ewg + 1), (ntiles - 1) & 1, abort_flag, err);
+      tc_fence_after();
+      named_bar_sync(3, 256);  // both warpgroups' contractions are complete: the stages may be reused
+#pragma unroll
+      for (int cc = 0; cc < D / 8; ++cc) {
+        uint32_t v0[8];
+        tmem_ld8(taddr(tbase, eq, ewg * C::T_STRIDE + C::T_S + 8 * cc), v0);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) stg[fr * (D + 1) + 8 * cc + k] = __uint_as_float(v0[k]);
+      }
+      stg[fr * (D + 1) + D] = zsum;
+      if (fvalid) part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + fr] = c_run;
+    } else {
     cw[ewg * 128 + frow] = c_run;
     cw[256 + ewg * 128 + frow] = zsum;
     named_bar_sync(3, 256);
     const int n0 = (ntiles + 1) / 2, n1 = ntiles / 2;  // tiles of each warpgroup
     const float c0 = cw[frow], c1 = cw[128 + frow];
     const float cmax = n1 > 0 ? fmaxf(c0, c1) : c0;
-    if (n0 > 0) mbar_wait(bar(C::B_SDONE + 0), (n0 - 1) & 1, abort_flag, err);
-    if (n1 > 0) mbar_wait(bar(C::B_SDONE + 1), (n1 - 1) & 1, abort_flag, err);
+    if (n0 > 0) mbar_wait(bar(C::B_SDONE + 1), (n0 - 1) & 1, abort_flag, err);
+    if (n1 > 0) mbar_wait(bar(C::B_SDONE + 3), (n1 - 1) & 1, abort_flag, err);
     tc_fence_after();
     const float s0 = n0 > 0 ? ex2(c0 - cmax) : 0.f, s1 = n1 > 0 ? ex2(c1 - cmax) : 0.f;
-    // the merged rows go through shared memory (the K stages are free now: every MMA has
-    // completed) so that the partial state is written with coalesced 16-byte stores; a row
-    // stride of D + 1 floats (odd) keeps the 32 rows of a warp on different banks
-    float* stg = reinterpret_cast<float*>(smem + C::S_K);
 #pragma unroll
     for (int cc = 0; cc < D / 16; ++cc) {  // this warpgroup's half of the columns
       const int col0 = ewg * (D / 2) + 8 * cc;
@@ -735,6 +788,7 @@ __global__ void __launch_bounds__(KeyPP::THREADS, 1) key_pass_pp_sm100(
     if (ewg == 0) {
       stg[frow * (D + 1) + D] = fmaf(cw[384 + frow], s1, cw[256 + frow] * s0);
       if (fvalid) part_c[(static_cast<size_t>(head) * P + p) * nsb + f0 + frow] = cmax;
+    }
     }
     named_bar_sync(3, 256);
     // this group's rows f0 .. f0 + gw - 1 are contiguous in the partial state; gw (D + 1) is a
@@ -1324,15 +1378,24 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   int rc = make_map(&mk, K, D, p.L, heads);
   if (rc == FAVOR_OK) rc = make_map(&mv, V, D, p.L, heads);
   if (rc != FAVOR_OK) return rc;
-  // d = 64: the two-warpgroup kernel; d = 128: the lock-step kernel
+  // d = 64: the two-warpgroup kernel (256 features per CTA when m > 128); d = 128: the lock-step kernel
   void (*kern)(const CUtensorMap, const CUtensorMap, const float*, float*, float*, int, int, int, int, int, float, float);
   int smem_bytes, threads;
+  const int nfeat = key_features_per_cta(p.d, p.m);
   if constexpr (D == 64) {
-    kern = key_pass_pp_sm100;
-    smem_bytes = KeyPP::SMEM;
-    threads = KeyPP::THREADS;
-    static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), threads);
-    if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), threads);
+    if (nfeat == 256) {
+      kern = key_pass_pp_sm100<true>;
+      smem_bytes = KeyPP<true>::SMEM;
+      threads = KeyPP<true>::THREADS;
+      static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), threads);
+      if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), threads);
+    } else {
+      kern = key_pass_pp_sm100<false>;
+      smem_bytes = KeyPP<false>::SMEM;
+      threads = KeyPP<false>::THREADS;
+      static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), threads);
+      if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), threads);
+    }
   } else {
     kern = key_pass_sm100<D>;
     smem_bytes = KeyCfg<D>::SMEM;
@@ -1341,7 +1404,7 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass attribute: %s", cudaGetErrorString(e));
   char* base = static_cast<char*>(partials);
-  dim3 grid((p.m + 127) / 128, p.P, heads);
+  dim3 grid((p.m + nfeat - 1) / nfeat, p.P, heads);
   e = launch_overlapped(kern, grid, dim3(threads), smem_bytes, st, overlap, mk, mv, W,
                         reinterpret_cast<float*>(base + p.part_S_off), reinterpret_cast<float*>(base + p.part_c_off),
                         p.L, p.m, p.P, p.chunk, p.nsb, p.wscale, p.nscale);
