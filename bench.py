@@ -454,7 +454,7 @@ def decode_entry(fv, dev, peaks, steps=400, graph_steps=100, T=256):
 
 def relu_entry(fv, dev, peaks, min_seconds=0.4):
     """Kernelizable attention with f = ReLU (favor_attention_relu) on the headline shape: ms per call,
-    with the path's roofline (fp32 FMA flops of both passes on the CUDA cores, or HBM bytes)."""
+    with the path's roofline (the bf16 tensor-core flops of both passes, or HBM bytes)."""
     w = wl.WORKLOADS["bf16_L16384_heavykeys"]
     Q, K, V = (t.to(dev) for t in wl.make_inputs(w))
     W = fv.favor_make_features(w.w_seed, w.m, w.d).to(dev)
@@ -484,15 +484,14 @@ def relu_entry(fv, dev, peaks, min_seconds=0.4):
     torch.cuda.synchronize(dev)
     fv.favor_device_check()
     ms = e0.elapsed_time(e1) / steps
-    G = w.H // w.Hkv
-    flops = w.units * (1 + 1 / G) * (2 * w.d * w.m + 2 * w.m * (w.d + 1))
-    hbm = w.units * 2 * (2 * w.d + 2 * w.d / G)
-    fma_pk = 2 * FFMA_PER_SM_CLK * NUM_SMS * peaks["sm_max_mhz"] * 1e6
-    t = {"fma": flops / fma_pk * 1e6, "hbm": hbm / (peaks["hbm_gbs"] * 1e9) * 1e6}
+    # bf16 with d = 64 runs on the tensor-core kernels with the map swapped: the same contractions
+    # and bytes as the exponential map, no exponentials (so no MUFU term)
+    rt = roofline_terms(w, peaks)
+    t = {"tensor": rt["t_tensor_us"], "hbm": rt["t_hbm_us"]}
     bound = max(t, key=t.get)
     return {"workload": w.name + "_relu", "feature_map": "relu", "dtype": "bf16", "steps": steps, "ms_per_step": ms,
             "value": whole_job_rate(w.units, 1, ms), "unit": UNIT,
-            "roofline_path": {"t_fma_us": t["fma"], "t_hbm_us": t["hbm"], "bound": bound,
+            "roofline_path": {"t_tensor_us": t["tensor"], "t_hbm_us": t["hbm"], "bound": bound,
                               "frac": t[bound] / (ms * 1e3)},
             "input_sets": len(sets)}
 

@@ -236,9 +236,14 @@ int relu_attention_impl(int dtype, const void* Q, const void* K, const void* V, 
   const size_t st_off = round_up(p.part_bytes, 256);
   FAVOR_CUDA_TRY(cudaMallocAsync(&ws, st_off + p.st_bytes, st), "favor_attention_relu scratch allocation");
   char* base = static_cast<char*>(ws);
-  int rc = simt_key_pass_relu(dtype, K, V, W, base, p, st);
+  // bf16 with d = 64: the tensor-core key pass with the map swapped; otherwise the CUDA-core one
+  int rc = dtype == FAVOR_BF16 && d == 64 ? sm100_key_pass_relu(K, V, W, base, p, st)
+                                          : simt_key_pass_relu(dtype, K, V, W, base, p, st);
   if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, p, st, false);
-  if (rc == FAVOR_OK) rc = simt_query_pass_relu(dtype, Q, W, base + st_off, out, p, st);
+  if (rc == FAVOR_OK)
+    rc = dtype == FAVOR_BF16 && d == 64 && m > 64 && m <= 512
+             ? sm100_query_pass_relu(Q, W, base + st_off, out, p, st)
+             : simt_query_pass_relu(dtype, Q, W, base + st_off, out, p, st);
   cudaError_t fe = cudaFreeAsync(ws, st);
   if (rc != FAVOR_OK) return rc;
   FAVOR_CUDA_TRY(fe, "favor_attention_relu scratch release");

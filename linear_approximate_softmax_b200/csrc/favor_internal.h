@@ -1,6 +1,7 @@
 // Internal declarations shared by the C-ABI layer and the kernels.
 #pragma once
 
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 
@@ -94,6 +95,12 @@ inline int key_features_per_cta(int d, int m) { return d == 64 && m > 128 ? 256 
 bool sm100_query_supported(const Plan& p);
 int sm100_key_pass(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st,
                    bool overlap);
+// The tensor-core key and query passes with the feature map f = ReLU (bf16, d = 64; the query
+// pass for 64 < m <= 512).
+int sm100_key_pass_relu(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st);
+int sm100_query_pass_relu(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st);
+// W's scale for the ReLU map: d^-1/4 (the exponential map's carries log2(e) as well).
+inline float relu_wscale(int d) { return static_cast<float>(1.0 / std::sqrt(std::sqrt(static_cast<double>(d)))); }
 int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,
                      bool overlap);
 // Reads and clears the device error word (bit 0: a bounded wait gave up).

@@ -497,8 +497,6 @@ int launch_linformer_query(const void* Q, const void* state, void* out, const Pl
   return FAVOR_OK;
 }
 
-// d^-1/4: the input scaling of the ReLU map (no log2(e): no exponential)
-float relu_wscale(int d) { return static_cast<float>(std::pow(static_cast<double>(d), -0.25)); }
 
 template <typename T, int D, int FMAP = kExp>
 int launch_key(const void* K, const void* V, const float* W, void* partials, const Plan& p,

@@ -450,7 +450,9 @@ struct KeyPP {
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-template <bool WIDE>
+// RELU: the feature map max(W'k, 0) instead of 2^(W'k - n(k) - c) (W' then carries no log2(e)): no
+// norms, no stabilisers (written as 0, so the reduction sums the chunks as they are), no rescale.
+template <bool WIDE, bool RELU>
 __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const float* __restrict__ W,
     float* __restrict__ part_S, float* __restrict__ part_c, int L, int m, int P, int chunk, int nsb, float wscale,
@@ -615,7 +617,7 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
     // shared-memory wavefront hit different banks.  The stage's norms are overwritten only after
     // the tile that last used it has been contracted, which needs its exponentials, which need
     // these norms, so no other wait is needed.
-    for (int i = 0; i < ntiles; ++i) {
+    for (int i = 0; i < (RELU ? 0 : ntiles); ++i) {
       const int s = i % C::NST;
       if (!mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err)) break;
 #pragma unroll 1
@@ -671,7 +673,7 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
           w2 = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, w2))));
         }
       }
-      floor_c = w2 * static_cast<float>(kLog2e * 0.5) - 64.f;
+      floor_c = RELU ? 0.f : w2 * static_cast<float>(kLog2e * 0.5) - 64.f;
     }
     float c_run = floor_c, tmax = -INFINITY, zsum = 0.f;  // zsum: this feature's normaliser sum_t phi
     const uint32_t cU = ewg * C::T_STRIDE + C::T_U, cP = ewg * C::T_STRIDE + C::T_P,
@@ -682,7 +684,7 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
       mbar_wait(bar(C::B_D1F + ewg), cnt & 1, abort_flag, err);
       // the norms of tile i (the norm warp cannot have moved on to the stage's next tile: that
       // tile is loaded only after this one has been contracted)
-      mbar_wait(bar(C::B_NRM + s), (i / C::NST) & 1, abort_flag, err);
+      if (!RELU) mbar_wait(bar(C::B_NRM + s), (i / C::NST) & 1, abort_flag, err);
       // this tile's U^T row into registers (one read), then release it to the next projection
       float ut[128];
 #pragma unroll
@@ -693,7 +695,7 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
       if (lane == 0) mbar_arrive(bar(C::B_UE + ewg));
       // the previous tile raised the running max: rescale S and the normaliser now, once the
       // previous tile's contraction is complete
-      const bool need = tmax > c_run + kTau;
+      const bool need = !RELU && tmax > c_run + kTau;
       if (__any_sync(0xffffffffu, need)) {
         if (cnt >= 1) mbar_wait(bar(C::B_SDONE + 2 * ewg + 1), (cnt - 1) & 1, abort_flag, err);
         tc_fence_after();
@@ -717,14 +719,21 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
         uint32_t wph[16];
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {  // two tokens per packed fp32x2 operation
-          const float4 n4 = nv[8 * q4 + k4];
           const float* r = &ut[32 * q4 + 4 * k4];
-          const float2 a01 = __fadd2_rn(make_float2(r[0], r[1]), make_float2(n4.x, n4.y));
-          const float2 a23 = __fadd2_rn(make_float2(r[2], r[3]), make_float2(n4.z, n4.w));
-          tm4[k4 & 3] = max3(tm4[k4 & 3], a01.x, a01.y);
-          tm4[k4 & 3] = max3(tm4[k4 & 3], a23.x, a23.y);
-          const float2 b01 = __fadd2_rn(a01, ncc), b23 = __fadd2_rn(a23, ncc);
-          const float2 p01 = make_float2(ex2(b01.x), ex2(b01.y)), p23 = make_float2(ex2(b23.x), ex2(b23.y));
+          float2 p01, p23;
+          if constexpr (RELU) {
+            p01 = make_float2(fmaxf(r[0], 0.f), fmaxf(r[1], 0.f));
+            p23 = make_float2(fmaxf(r[2], 0.f), fmaxf(r[3], 0.f));
+          } else {
+            const float4 n4 = nv[8 * q4 + k4];
+            const float2 a01 = __fadd2_rn(make_float2(r[0], r[1]), make_float2(n4.x, n4.y));
+            const float2 a23 = __fadd2_rn(make_float2(r[2], r[3]), make_float2(n4.z, n4.w));
+            tm4[k4 & 3] = max3(tm4[k4 & 3], a01.x, a01.y);
+            tm4[k4 & 3] = max3(tm4[k4 & 3], a23.x, a23.y);
+            const float2 b01 = __fadd2_rn(a01, ncc), b23 = __fadd2_rn(a23, ncc);
+            p01 = make_float2(ex2(b01.x), ex2(b01.y));
+            p23 = make_float2(ex2(b23.x), ex2(b23.y));
+          }
           zs2 = __fadd2_rn(zs2, __fadd2_rn(p01, p23));
           wph[2 * k4] = pack_bf16x2(p01.x, p01.y);
           wph[2 * k4 + 1] = pack_bf16x2(p23.x, p23.y);
@@ -1372,7 +1381,7 @@ int check_register_split(const void* kern, int threads, long need = -1) {
 
 template <int D>
 int launch_key(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st,
-               bool overlap) {
+               bool overlap, bool relu = false) {
   CUtensorMap mk, mv;
   const int heads = p.B * p.Hkv;
   int rc = make_map(&mk, K, D, p.L, heads);
@@ -1383,20 +1392,22 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   int smem_bytes, threads;
   const int nfeat = key_features_per_cta(p.d, p.m);
   if constexpr (D == 64) {
-    if (nfeat == 256) {
-      kern = key_pass_pp_sm100<true>;
-      smem_bytes = KeyPP<true>::SMEM;
-      threads = KeyPP<true>::THREADS;
-      static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), threads);
-      if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), threads);
-    } else {
-      kern = key_pass_pp_sm100<false>;
-      smem_bytes = KeyPP<false>::SMEM;
-      threads = KeyPP<false>::THREADS;
-      static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), threads);
-      if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), threads);
-    }
+    // each variant's register split is checked once
+    static const int split[4] = {
+        check_register_split(reinterpret_cast<const void*>(key_pass_pp_sm100<false, false>), KeyPP<false>::THREADS),
+        check_register_split(reinterpret_cast<const void*>(key_pass_pp_sm100<true, false>), KeyPP<true>::THREADS),
+        check_register_split(reinterpret_cast<const void*>(key_pass_pp_sm100<false, true>), KeyPP<false>::THREADS),
+        check_register_split(reinterpret_cast<const void*>(key_pass_pp_sm100<true, true>), KeyPP<true>::THREADS)};
+    const bool wide = nfeat == 256;
+    kern = wide ? (relu ? key_pass_pp_sm100<true, true> : key_pass_pp_sm100<true, false>)
+                : (relu ? key_pass_pp_sm100<false, true> : key_pass_pp_sm100<false, false>);
+    smem_bytes = wide ? KeyPP<true>::SMEM : KeyPP<false>::SMEM;
+    threads = KeyPP<true>::THREADS;
+    const int v = (relu ? 2 : 0) + (wide ? 1 : 0);
+    if (split[v] != FAVOR_OK)
+      return check_register_split(reinterpret_cast<const void*>(kern), threads);
   } else {
+    if (relu) return set_error(FAVOR_ERR_UNSUPPORTED, "sm100 key pass: the ReLU map needs d = 64");
     kern = key_pass_sm100<D>;
     smem_bytes = KeyCfg<D>::SMEM;
     threads = kThreads;
@@ -1407,7 +1418,7 @@ int launch_key(const void* K, const void* V, const float* W, void* partials, con
   dim3 grid((p.m + nfeat - 1) / nfeat, p.P, heads);
   e = launch_overlapped(kern, grid, dim3(threads), smem_bytes, st, overlap, mk, mv, W,
                         reinterpret_cast<float*>(base + p.part_S_off), reinterpret_cast<float*>(base + p.part_c_off),
-                        p.L, p.m, p.P, p.chunk, p.nsb, p.wscale, p.nscale);
+                        p.L, p.m, p.P, p.chunk, p.nsb, relu ? relu_wscale(p.d) : p.wscale, p.nscale);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 key pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
 }
@@ -1436,7 +1447,7 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
 }
 
 int launch_query_d64(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,
-                     bool overlap) {
+                     bool overlap, bool relu = false) {
   using C = QueryD64;
   CUtensorMap mq, mo;
   const int bh = p.B * p.H;
@@ -1444,17 +1455,20 @@ int launch_query_d64(const void* Q, const float* W, const void* state, void* out
   if (rc == FAVOR_OK) rc = make_map(&mo, out, C::D, p.L, bh, 32);  // stored by each output warp, 32 rows
   if (rc != FAVOR_OK) return rc;
   if (p.op_rows != C::NROWS) return set_error(FAVOR_ERR_UNSUPPORTED, "query pass: state image without the normaliser rows");
-  auto kern = query_pass_d64_sm100;
+  auto kern = relu ? query_pass_d64_sm100<true> : query_pass_d64_sm100<false>;
   const long need = 128L * C::R_CTL + 128L * C::R_CVT + 256L * C::R_EPI;
-  static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), C::THREADS, need);
-  if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), C::THREADS, need);
+  static const int split_ok[2] = {
+      check_register_split(reinterpret_cast<const void*>(query_pass_d64_sm100<false>), C::THREADS, need),
+      check_register_split(reinterpret_cast<const void*>(query_pass_d64_sm100<true>), C::THREADS, need)};
+  if (split_ok[relu ? 1 : 0] != FAVOR_OK)
+    return check_register_split(reinterpret_cast<const void*>(kern), C::THREADS, need);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass attribute: %s", cudaGetErrorString(e));
   const int ntiles = bh * ((p.L + 127) / 128);
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
   const unsigned char* img = static_cast<const unsigned char*>(state) + p.st_op_off;
   e = launch_overlapped(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, overlap, mq, mo, W, img, p.L, p.m, p.H,
-                        p.Hkv, ntiles, static_cast<int>(p.op_bytes), p.wscale);
+                        p.Hkv, ntiles, static_cast<int>(p.op_bytes), relu ? relu_wscale(p.d) : p.wscale);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
 }
@@ -1472,6 +1486,17 @@ int sm100_key_pass(const void* K, const void* V, const float* W, void* partials,
                    bool overlap) {
   return p.d == 64 ? launch_key<64>(K, V, W, partials, p, st, overlap)
                    : launch_key<128>(K, V, W, partials, p, st, overlap);
+}
+
+int sm100_query_pass_relu(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st) {
+  if (!(p.d == 64 && p.m > 64 && p.m <= QueryD64::MMAX))
+    return set_error(FAVOR_ERR_UNSUPPORTED, "sm100 query pass: the ReLU map needs d = 64 and 64 < m <= 512");
+  return launch_query_d64(Q, W, state, out, p, st, false, true);
+}
+
+int sm100_key_pass_relu(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st) {
+  if (p.d != 64) return set_error(FAVOR_ERR_UNSUPPORTED, "sm100 key pass: the ReLU map needs d = 64");
+  return launch_key<64>(K, V, W, partials, p, st, false, true);
 }
 
 int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,

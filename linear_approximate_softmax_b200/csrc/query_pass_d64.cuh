@@ -68,6 +68,10 @@ struct QueryD64 {
   static_assert(S_SP % 1024 == 0 && S_Q % 1024 == 0 && S_STG % 1024 == 0, "swizzled operands on 1024-byte boundaries");
 };
 
+// RELU: the feature map max(W'q, 0) (W' then carries no log2(e)).  The image's exponents e_f become
+// factors 2^e_f once the image is in (zero past m), and phi' = max(U, 0) 2^k 2^e_f 2^-c with an
+// integer row stabiliser c that keeps phi' below 2^15, raised like the exponential map's.
+template <bool RELU>
 __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, const float* __restrict__ W,
     const unsigned char* __restrict__ op_img, int L, int m, int H, int Hkv, int ntiles_total, int op_bytes,
@@ -194,6 +198,11 @@ __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
           }
           if (!mbar_wait<true>(bar(C::B_SF), k & 1, abort_flag, err)) break;
           inflight = false;
+          if constexpr (RELU) {  // e_f -> 2^e_f in place (the next image's copy is ordered after this)
+            float* ef = reinterpret_cast<float*>(smem + C::S_SP + C::NROWS * 128 * nb);
+            for (int f = 0; f < nb * C::FB; ++f) ef[f] = ex2(ef[f]);
+            fence_proxy_async_smem();
+          }
           st_release_shared(img_count, k + 1);
         }
         if (inflight) mbar_wait(bar(C::B_SF), k & 1, abort_flag, err, 200000000ull);  // drain after a failure
@@ -324,6 +333,38 @@ __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
             ph[k2] = pack_f16x2(ex2(bb.x), ex2(bb.y));
           }
         };
+        if constexpr (RELU) {
+          // t = max(U, 0) 2^k 2^e_f and its maximum; phi' = t 2^-c
+#pragma unroll
+          for (int k4 = 0; k4 < C::FB / 4; ++k4) {
+            const float4 s4 = e4p[k4];  // 2^e_f
+            v[4 * k4 + 0] = fmaxf(v[4 * k4 + 0], 0.f) * (up * s4.x);
+            v[4 * k4 + 1] = fmaxf(v[4 * k4 + 1], 0.f) * (up * s4.y);
+            v[4 * k4 + 2] = fmaxf(v[4 * k4 + 2], 0.f) * (up * s4.z);
+            v[4 * k4 + 3] = fmaxf(v[4 * k4 + 3], 0.f) * (up * s4.w);
+            m4[k4 & 3] = fmax3(m4[k4 & 3], v[4 * k4 + 0], v[4 * k4 + 1]);
+            m4[k4 & 3] = fmax3(m4[k4 & 3], v[4 * k4 + 2], v[4 * k4 + 3]);
+          }
+          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          // the integer c = E(mx) - 14 puts the block's largest phi' in [2^14, 2^15) (a row of zeros keeps c)
+          const int cm = mx > 0.f ? ((__float_as_int(mx) >> 23) & 0xFF) - 127 - 14 : -1000;
+          if (j == 0) {
+            c = mx > 0.f ? static_cast<float>(max(-120, min(120, cm))) : 0.f;
+          } else {
+            const bool need = cm > static_cast<int>(c);
+            if (__any_sync(0xffffffffu, need)) {  // cold: raise c for those rows, rescale the contractions so far
+              mbar_wait(bar(C::B_M2 + 2 * w + ((b - 1) & 1)), ((b - 1) >> 1) & 1, abort_flag, err);
+              tc_fence_after();
+              const int cn = need ? min(120, cm) : static_cast<int>(c);
+              scale_tmem_row(taddr(tbase, eq, cO), C::NROWS / 8,
+                             __int_as_float((127 + max(-126, static_cast<int>(c) - cn)) << 23));
+              c = static_cast<float>(cn);
+            }
+          }
+          const float rc = __int_as_float((127 - static_cast<int>(c)) << 23);  // 2^-c
+#pragma unroll
+          for (int k2 = 0; k2 < C::FB / 2; ++k2) ph[k2] = pack_f16x2(v[2 * k2] * rc, v[2 * k2 + 1] * rc);
+        } else
         // v = 2^k U + e (a feature past m has W' = 0 and e = -inf: v = -inf), and its maximum
         if (j == 0) {  // the row's first block: its exact maximum first, then the exponentials
 #pragma unroll
@@ -406,7 +447,9 @@ __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
       if (lane == 0) mbar_arrive(bar(C::B_QE + s));  // this warp has read its rows of the stage
       // the biased bf16 exponent of the row's largest |q|
       const int ebits = static_cast<int>(max(emax & 0xFFFFu, emax >> 16) >> 7);
-      const int k = min(100, max(0, ebits - 141));
+      // the ReLU map is scale-free per row, so its small rows are scaled up as well (a row of zeros
+      // keeps k = -100 and stays zero)
+      const int k = min(100, max(RELU ? -100 : 0, ebits - 141));
       const bool plain = __all_sync(0xffffffffu, k == 0);
       const float down = __int_as_float((127 - k) << 23);
       uint32_t o[32];

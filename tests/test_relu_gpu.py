@@ -72,3 +72,21 @@ def test_relu_full_size_headline_shape_every_element(parity_report):
     w = wl.WORKLOADS["bf16_L16384_heavykeys"]
     Q, K, V = wl.make_inputs(w)
     run_relu(Q, K, V, w.m, w.w_seed, True, f"{w.name} full size", parity_report)
+
+
+def test_relu_query_rows_scaled_by_powers_of_two():
+    # phi(c q) = c phi(q) for c > 0, so each query row's output does not depend on its scale.  Rows
+    # scaled by 2^-30 .. 2^30 (exact in bf16) drive the tensor-core query pass's integer row
+    # stabiliser over its whole range, including raises after a row's first feature block.
+    Q, K, V = wl.random_inputs(1, 4, 2, 600, 64, torch.bfloat16, seed=91)
+    rng = np.random.default_rng(5)
+    e = torch.from_numpy(rng.integers(-30, 31, size=(1, 4, 600, 1)).astype(np.float32))
+    Qs = (Q.float() * torch.exp2(e)).to(torch.bfloat16)
+    assert torch.equal(Qs.float(), Q.float() * torch.exp2(e))
+    for m in (128, 256, 512):
+        run_relu(Qs, K, V, m, what=f"rows scaled by 2^-30..2^30, m={m}")
+        W = fv.favor_make_features(1, m, 64).cuda()
+        a = fv.favor_attention_relu(Qs.cuda(), K.cuda(), V.cuda(), W).float()
+        b = fv.favor_attention_relu(Q.cuda(), K.cuda(), V.cuda(), W).float()
+        fv.favor_device_check()
+        assert (a - b).abs().max().item() <= 2e-2, m
