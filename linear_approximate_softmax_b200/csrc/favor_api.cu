@@ -266,7 +266,9 @@ int linformer_impl(int dtype, const void* Q, const void* K, const void* V, const
   char* base = static_cast<char*>(ws);
   int rc = simt_linformer_proj(dtype, K, V, E, F, base, pk, B * Hkv, st);
   if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, pk, st, false);
-  if (rc == FAVOR_OK) rc = simt_linformer_query(dtype, Q, base + st_off, out, pq, pk, st);
+  if (rc == FAVOR_OK)
+    rc = dtype == FAVOR_BF16 && d == 64 && kp > 64 && kp <= 512 ? sm100_linformer_query(Q, base + st_off, out, pq, pk, st)
+                                                               : simt_linformer_query(dtype, Q, base + st_off, out, pq, pk, st);
   cudaError_t fe = cudaFreeAsync(ws, st);
   if (rc != FAVOR_OK) return rc;
   FAVOR_CUDA_TRY(fe, "favor_linformer scratch release");

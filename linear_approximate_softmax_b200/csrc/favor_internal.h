@@ -99,6 +99,9 @@ int sm100_key_pass(const void* K, const void* V, const float* W, void* partials,
 // pass for 64 < m <= 512).
 int sm100_key_pass_relu(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st);
 int sm100_query_pass_relu(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st);
+// Linformer's projected query pass on the tensor cores (bf16, d = 64, 64 < k <= 512): the query
+// pass of each kv head with its projected keys as W and its projected values as the state.
+int sm100_linformer_query(const void* Q, const void* state, void* out, const Plan& pq, const Plan& pk, cudaStream_t st);
 // W's scale for the ReLU map: d^-1/4 (the exponential map's carries log2(e) as well).
 inline float relu_wscale(int d) { return static_cast<float>(1.0 / std::sqrt(std::sqrt(static_cast<double>(d)))); }
 int sm100_query_pass(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,

@@ -1446,8 +1446,9 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   return FAVOR_OK;
 }
 
-int launch_query_d64(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,
-                     bool overlap, bool relu = false) {
+// img: the state images of the plan's kv heads; W: m rows of d floats, w_row floats apart
+int launch_query_d64_img(const void* Q, const float* W, int w_row, float wscale, const unsigned char* img, void* out,
+                         const Plan& p, cudaStream_t st, bool overlap, bool relu) {
   using C = QueryD64;
   CUtensorMap mq, mo;
   const int bh = p.B * p.H;
@@ -1466,11 +1467,16 @@ int launch_query_d64(const void* Q, const float* W, const void* state, void* out
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass attribute: %s", cudaGetErrorString(e));
   const int ntiles = bh * ((p.L + 127) / 128);
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
-  const unsigned char* img = static_cast<const unsigned char*>(state) + p.st_op_off;
   e = launch_overlapped(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, overlap, mq, mo, W, img, p.L, p.m, p.H,
-                        p.Hkv, ntiles, static_cast<int>(p.op_bytes), relu ? relu_wscale(p.d) : p.wscale);
+                        p.Hkv, ntiles, static_cast<int>(p.op_bytes), wscale, w_row);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
+}
+
+int launch_query_d64(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st,
+                     bool overlap, bool relu = false) {
+  return launch_query_d64_img(Q, W, p.d, relu ? relu_wscale(p.d) : p.wscale,
+                              static_cast<const unsigned char*>(state) + p.st_op_off, out, p, st, overlap, relu);
 }
 
 }  // namespace
@@ -1486,6 +1492,29 @@ int sm100_key_pass(const void* K, const void* V, const float* W, void* partials,
                    bool overlap) {
   return p.d == 64 ? launch_key<64>(K, V, W, partials, p, st, overlap)
                    : launch_key<128>(K, V, W, partials, p, st, overlap);
+}
+
+int sm100_linformer_query(const void* Q, const void* state, void* out, const Plan& pq, const Plan& pk, cudaStream_t st) {
+  if (!(pq.d == 64 && pq.m > 64 && pq.m <= QueryD64::MMAX))
+    return set_error(FAVOR_ERR_UNSUPPORTED, "sm100 projected query: needs d = 64 and 64 < k <= 512");
+  // one launch per kv head t: its G query heads (b H + h G .. + G - 1 = G t ..) are contiguous, its
+  // projected keys d^-1/4 E K are the state rows of head B Hkv + t (rows d + 1 floats apart) and F V
+  // is the state image of head t
+  const int heads = pq.B * pq.Hkv, G = pq.H / pq.Hkv, D1 = pq.d + 1;
+  Plan p1;
+  int rc = make_plan(1, G, 1, pq.L, pq.d, pq.m, &p1);
+  if (rc != FAVOR_OK) return rc;
+  const float* S = reinterpret_cast<const float*>(static_cast<const char*>(state) + pk.st_S_off);
+  const unsigned char* img = static_cast<const unsigned char*>(state) + pk.st_op_off;
+  const size_t qstride = static_cast<size_t>(G) * pq.L * pq.d * 2;  // bytes of bf16 per kv head's queries
+  for (int t = 0; t < heads && rc == FAVOR_OK; ++t)
+    // the first launch reads the reduction's output before any wait: an ordinary launch; later ones
+    // follow query launches, which write only their own output rows
+    rc = launch_query_d64_img(static_cast<const char*>(Q) + t * qstride,
+                              S + (static_cast<size_t>(heads) + t) * pq.m * D1, D1, pq.wscale,
+                              img + static_cast<size_t>(t) * pk.op_bytes, static_cast<char*>(out) + t * qstride, p1, st,
+                              t > 0, false);
+  return rc;
 }
 
 int sm100_query_pass_relu(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st) {

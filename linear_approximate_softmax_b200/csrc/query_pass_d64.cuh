@@ -75,7 +75,7 @@ template <bool RELU>
 __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, const float* __restrict__ W,
     const unsigned char* __restrict__ op_img, int L, int m, int H, int Hkv, int ntiles_total, int op_bytes,
-    float wscale) {
+    float wscale, int w_row) {
   using C = QueryD64;
   constexpr int NQS = C::NQS;
   extern __shared__ unsigned char smem_raw[];
@@ -145,10 +145,10 @@ __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       float w0 = 0.f, w1 = 0.f;
-      if (f < m) {
-        const float2 v = *reinterpret_cast<const float2*>(W + static_cast<size_t>(f) * C::D + 8 * c + 2 * k);
-        w0 = v.x * wscale;
-        w1 = v.y * wscale;
+      if (f < m) {  // row f of W starts at f * w_row floats (w_row >= D, possibly odd)
+        const float* wr = W + static_cast<size_t>(f) * w_row + 8 * c + 2 * k;
+        w0 = wr[0] * wscale;
+        w1 = wr[1] * wscale;
       }
       h[k] = pack_f16x2(w0, w1);
     }
