@@ -498,7 +498,7 @@ def relu_entry(fv, dev, peaks, min_seconds=0.4):
 
 def linformer_entry(fv, dev, peaks, kp=256, min_seconds=0.4):
     """Linformer projected attention (favor_linformer) on the headline shape with k = 256 projected
-    rows: ms per call, with the path's roofline (the projections' fp32 FMA flops, then the attention
+    rows: ms per call, with the path's roofline (the projections' bf16 tensor flops, then the attention
     over k on the tensor cores and the MUFU; or HBM bytes of Q, K, V, out, E and F)."""
     w = wl.WORKLOADS["bf16_L16384_heavykeys"]
     Q, K, V = (t.to(dev) for t in wl.make_inputs(w))
@@ -531,25 +531,25 @@ def linformer_entry(fv, dev, peaks, kp=256, min_seconds=0.4):
     torch.cuda.synchronize(dev)
     fv.favor_device_check()
     ms = e0.elapsed_time(e1) / steps
-    # the projections E K and F V run on the CUDA cores (fp32 FMA); the attention over the k projected
-    # rows runs on the tensor cores (bf16 flops) and the MUFU (exponentials).  The two are separate
-    # kernels, one after the other, so the path's bound is the projections' time plus the attention's.
+    # the projections E K and F V (bf16 tensor flops) and the attention over the k projected rows
+    # (tensor flops and MUFU exponentials) are separate kernels, one after the other, so the path's
+    # bound is the projections' time plus the attention's.
     kv_heads, q_heads = w.B * w.Hkv, w.B * w.H
     clk = peaks["sm_max_mhz"] * 1e6
     proj_flops = kv_heads * 2 * (2 * kp * w.L * w.d)
     att_flops = q_heads * w.L * (2 * kp * w.d + 2 * kp * (w.d + 1))
     exps = q_heads * w.L * kp
     hbm = w.units * 2 * (2 * w.d + 2 * w.d * w.Hkv / w.H) + 2 * kp * w.L * 4
-    t = {"proj_fma": proj_flops / (2 * FFMA_PER_SM_CLK * NUM_SMS * clk) * 1e6,
+    t = {"proj_tensor": proj_flops / (peaks["bf16_tflops"] * 1e12) * 1e6,
          "att_tensor": att_flops / (peaks["bf16_tflops"] * 1e12) * 1e6,
          "att_mufu": exps / (MUFU_PER_SM_CLK * NUM_SMS * clk) * 1e6,
          "hbm": hbm / (peaks["hbm_gbs"] * 1e9) * 1e6}
-    bound_us = max(t["proj_fma"] + max(t["att_tensor"], t["att_mufu"]), t["hbm"])
+    bound_us = max(t["proj_tensor"] + max(t["att_tensor"], t["att_mufu"]), t["hbm"])
     return {"workload": w.name + "_linformer_k256", "dtype": "bf16", "kp": kp, "steps": steps, "ms_per_step": ms,
             "value": whole_job_rate(w.units, 1, ms), "unit": UNIT,
-            "roofline_path": {"t_proj_fma_us": t["proj_fma"], "t_att_tensor_us": t["att_tensor"],
+            "roofline_path": {"t_proj_tensor_us": t["proj_tensor"], "t_att_tensor_us": t["att_tensor"],
                               "t_att_mufu_us": t["att_mufu"], "t_hbm_us": t["hbm"],
-                              "bound": "projections (fp32 FMA) + attention (slower of tensor and MUFU)",
+                              "bound": "projections (tensor) + attention (slower of tensor and MUFU)",
                               "bound_us": bound_us, "frac": bound_us / (ms * 1e3)},
             "input_sets": len(sets)}
 

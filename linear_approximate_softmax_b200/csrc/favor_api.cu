@@ -2,6 +2,7 @@
 // Every exported function is declared and documented in include/favor.h.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -136,9 +137,13 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
 void plan_limit_chunks(Plan* p, int max_P) {
   if (max_P < 1) max_P = 1;
   if (p->P <= max_P) return;
+  plan_set_chunks(p, max_P);
+}
+
+void plan_set_chunks(Plan* p, int P) {
   const int heads = p->B * p->Hkv;
   const int tiles = (p->L + kTileTokens - 1) / kTileTokens;
-  const int chunk_tiles = (tiles + max_P - 1) / max_P;
+  const int chunk_tiles = (tiles + std::max(1, std::min(P, tiles)) - 1) / std::max(1, std::min(P, tiles));
   p->chunk = chunk_tiles * kTileTokens;
   p->P = (tiles + chunk_tiles - 1) / chunk_tiles;
   const size_t D1 = static_cast<size_t>(p->d) + 1;
@@ -259,12 +264,24 @@ int linformer_impl(int dtype, const void* Q, const void* K, const void* V, const
   Plan pq, pk;
   FAVOR_TRY(make_plan(B, H, Hkv, L, d, kp, &pq));
   FAVOR_TRY(make_plan(2 * B, H, Hkv, L, d, kp, &pk));  // the projected keys ride as B more batches
+  // bf16 with d = 64: the projections on the tensor cores, in enough key chunks for about six
+  // waves of CTAs (128 projected rows x chunk x product each)
+  const bool tc = dtype == FAVOR_BF16 && d == 64;
+  if (tc) {
+    int sms = 0;
+    FAVOR_TRY(device_sm_count(&sms));
+    const long per_chunk = static_cast<long>((kp + 127) / 128) * 2 * B * Hkv;
+    plan_set_chunks(&pk, static_cast<int>(std::max(1L, (6L * sms + per_chunk - 1) / per_chunk)));
+  }
   keep_pool_mapped();
   void* ws = nullptr;
   const size_t st_off = round_up(pk.part_bytes, 256);
-  FAVOR_CUDA_TRY(cudaMallocAsync(&ws, st_off + pk.st_bytes, st), "favor_linformer scratch allocation");
+  const size_t split_off = st_off + round_up(pk.st_bytes, 256);
+  const size_t ws_bytes = split_off + (tc ? linformer_split_bytes(kp, L) : 0);
+  FAVOR_CUDA_TRY(cudaMallocAsync(&ws, ws_bytes, st), "favor_linformer scratch allocation");
   char* base = static_cast<char*>(ws);
-  int rc = simt_linformer_proj(dtype, K, V, E, F, base, pk, B * Hkv, st);
+  int rc = tc ? sm100_linformer_proj(K, V, E, F, base + split_off, base, pk, B * Hkv, st)
+              : simt_linformer_proj(dtype, K, V, E, F, base, pk, B * Hkv, st);
   if (rc == FAVOR_OK) rc = run_reduce(base, base + st_off, pk, st, false);
   if (rc == FAVOR_OK)
     rc = dtype == FAVOR_BF16 && d == 64 && kp > 64 && kp <= 512 ? sm100_linformer_query(Q, base + st_off, out, pq, pk, st)

@@ -53,6 +53,8 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p);
 // Re-splits the key pass of `p` into at most max_P chunks per kv head and
 // recomputes the partials layout (the state layout does not depend on it).
 void plan_limit_chunks(Plan* p, int max_P);
+// Re-splits the key chunks into P of them (as near as whole 128-token tiles allow).
+void plan_set_chunks(Plan* p, int P);
 
 // The three steps of the path, each dispatched to its kernel on `st`.  overlap: launch the
 // kernel so that it may start while the kernel before it on `st` finishes (it waits before it
@@ -99,6 +101,11 @@ int sm100_key_pass(const void* K, const void* V, const float* W, void* partials,
 // pass for 64 < m <= 512).
 int sm100_key_pass_relu(const void* K, const void* V, const float* W, void* partials, const Plan& p, cudaStream_t st);
 int sm100_query_pass_relu(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st);
+// Linformer's projections E K and F V on the tensor cores (d = 64): E and F split into bf16 hi + lo
+// in `split` (linformer_split_bytes), then the partial states of the plan's 2 heads kv heads.
+size_t linformer_split_bytes(int kp, int L);
+int sm100_linformer_proj(const void* K, const void* V, const float* E, const float* F, void* split, void* partials,
+                         const Plan& pk, int heads, cudaStream_t st);
 // Linformer's projected query pass on the tensor cores (bf16, d = 64, 64 < k <= 512): the query
 // pass of each kv head with its projected keys as W and its projected values as the state.
 int sm100_linformer_query(const void* Q, const void* state, void* out, const Plan& pq, const Plan& pk, cudaStream_t st);

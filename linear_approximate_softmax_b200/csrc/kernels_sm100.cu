@@ -813,6 +813,156 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
 }
 
 // ============================================================================
+// Linformer projections on the tensor cores (d = 64, bf16 K and V)
+// ============================================================================
+// Linformer notes page, "4 Model": E K and F V (k x d per kv head).  E and F (fp32) are first
+// split into bf16 hi + lo (hi = bf16(x), lo = bf16(x - hi): about 16 bits of x).  One CTA takes a
+// (128 projected rows, key chunk, product) and accumulates (Ehi + Elo)[rows, chunk] K[chunk, :]
+// in tensor memory (M = 128, N = 64, 16 tokens per MMA; the E tile K-major, the K tile MN-major,
+// both as loaded), then writes the key pass's partial-state layout: F V with the constant column
+// 1 on chunk 0 only (the reduction's sum is then 1) as head h, d^-1/4 E K as head heads + h,
+// every stabiliser 0.
+struct LinProj {
+  static constexpr int D = 64;
+  // warp 0 TMA producer, warp 1 MMA issuer, warps 2-5 epilogue (TMEM lane quarter = warp % 4)
+  static constexpr int THREADS = 192;
+  static constexpr int NST = 4;                  // stages of TT tokens
+  static constexpr int TT = 64;
+  static constexpr int A_TILE = 128 * TT * 2;    // 128 rows x 64 tokens, bf16, K-major SW128
+  static constexpr int B_TILE = TT * D * 2;      // 64 tokens x 64 dims, bf16, MN-major SW128
+  static constexpr int STAGE = 2 * A_TILE + B_TILE;  // E hi, E lo, K (or F hi, F lo, V)
+  static constexpr int S_BAR = NST * STAGE;
+  static constexpr int B_FULL = 0, B_EMPTY = NST, B_DONE = 2 * NST, NBAR = 2 * NST + 1;
+  static constexpr int S_TPTR = S_BAR + NBAR * 8;
+  static constexpr int S_ABORT = S_TPTR + 8;
+  static constexpr int SMEM = S_ABORT + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(A_TILE % 1024 == 0 && B_TILE % 1024 == 0, "swizzled operands on 1024-byte boundaries");
+};
+
+// [4][kpad][Lpad] bf16: E hi, E lo, F hi, F lo; rows kp .. kpad - 1 and tokens L .. Lpad - 1 are zero
+// (Lpad, a multiple of 64, gives the rows the 16-byte stride a tensor map needs)
+__global__ void split_hi_lo_kernel(const float* __restrict__ E, const float* __restrict__ F,
+                                   __nv_bfloat16* __restrict__ out, int kp, int kpad, int L, int Lpad) {
+  const size_t n = static_cast<size_t>(kpad) * Lpad;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int j = static_cast<int>(i / Lpad), t = static_cast<int>(i - static_cast<size_t>(j) * Lpad);
+    const bool valid = j < kp && t < L;
+    const size_t src = static_cast<size_t>(j) * L + t;
+    const float e = valid ? E[src] : 0.f, f = valid ? F[src] : 0.f;
+    const __nv_bfloat16 eh = __float2bfloat16_rn(e), fh = __float2bfloat16_rn(f);
+    out[i] = eh;
+    out[n + i] = __float2bfloat16_rn(e - __bfloat162float(eh));
+    out[2 * n + i] = fh;
+    out[3 * n + i] = __float2bfloat16_rn(f - __bfloat162float(fh));
+  }
+}
+
+__global__ void __launch_bounds__(LinProj::THREADS, 1) linformer_proj_sm100(
+    const __grid_constant__ CUtensorMap tmEF, const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV, float* __restrict__ part_S, float* __restrict__ part_c, int L, int kp,
+    int P, int chunk, int nsb, int heads, float kscale) {
+  using C = LinProj;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int mt = blockIdx.x, p = blockIdx.y, z = blockIdx.z;
+  const bool isE = z >= heads;  // E K of kv head z - heads, or F V of kv head z
+  const int head = isE ? z - heads : z;
+  const int t_begin = p * chunk, t_end = min(L, t_begin + chunk);
+  const int ntiles = (t_end - t_begin + C::TT - 1) / C::TT;  // chunk is a multiple of TT: only L cuts a stage
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
+  uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
+  auto bar = [&](int i) { return sbase + C::S_BAR + 8u * i; };
+  unsigned int* err = &g_sm100_error_word;
+  const int zs = isE ? 0 : 2;  // E hi, E lo at split index 0, 1; F at 2, 3
+  const CUtensorMap* tmB = isE ? &tmK : &tmV;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(bar(C::B_FULL + s), 1);
+      mbar_init(bar(C::B_EMPTY + s), 1);
+    }
+    mbar_init(bar(C::B_DONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmEF);
+    prefetch_tmap(tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tptr_slot), 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tptr_slot;
+  griddep_wait();  // the split of E and F is the kernel before this one
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---------------- TMA producer ----------------
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % C::NST;
+        if (i >= C::NST && !mbar_wait<true>(bar(C::B_EMPTY + s), ((i / C::NST) - 1) & 1, abort_flag, err)) break;
+        const int t0 = t_begin + C::TT * i;
+        const uint32_t st = sbase + s * C::STAGE;
+        mbar_arrive_expect_tx(bar(C::B_FULL + s), C::STAGE);
+        tma_load_3d(st, &tmEF, bar(C::B_FULL + s), t0, 128 * mt, zs);  // x = token, y = row, z = split
+        tma_load_3d(st + C::A_TILE, &tmEF, bar(C::B_FULL + s), t0, 128 * mt, zs + 1);
+        tma_load_3d(st + 2 * C::A_TILE, tmB, bar(C::B_FULL + s), 0, t0, head);  // x = dim, y = token, z = head
+        issued = i + 1;
+      }
+      for (int i = max(0, issued - C::NST); i < issued; ++i)  // no copy is in flight when the CTA leaves
+        mbar_wait(bar(C::B_FULL + i % C::NST), (i / C::NST) & 1, abort_flag, err, 200000000ull);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---------------- MMA issuer ----------------
+      const uint32_t idesc = idesc_bf16(128, C::D, false, true);
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % C::NST;
+        if (!mbar_wait(bar(C::B_FULL + s), (i / C::NST) & 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t st = sbase + s * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < C::TT / 16; ++kk) {  // 16 tokens per step: Ehi then Elo against the same K rows
+          const uint64_t bd = sdesc_sw128(st + 2 * C::A_TILE + 2048 * kk, 16, 1024);
+          mma_ss(tbase, sdesc_sw128(st + 32 * kk, 16, 1024), bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ss(tbase, sdesc_sw128(st + C::A_TILE + 32 * kk, 16, 1024), bd, idesc, 1u);
+        }
+        mma_commit(bar(C::B_EMPTY + s));
+      }
+      mma_commit(bar(C::B_DONE));  // arrives once every MMA above has completed
+    }
+  } else {  // ---------------- epilogue: one projected row per thread ----------------
+    const int eq = warp & 3;
+    const int r = eq * 32 + lane, j = 128 * mt + r;
+    const bool ok = mbar_wait(bar(C::B_DONE), 0, abort_flag, err, 200000000ull);
+    tc_fence_after();
+    uint32_t acc[64];
+    tmem_ld32(taddr(tbase, eq, 0), *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
+    tmem_ld32(taddr(tbase, eq, 32), *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
+    tmem_wait_ld();
+    if (j < kp) {
+      float* out = part_S + (static_cast<size_t>(z) * P + p) * static_cast<size_t>(kp) * (C::D + 1) +
+                   static_cast<size_t>(j) * (C::D + 1);
+      const float sc = isE ? kscale : 1.f;
+      const bool any = ok && ntiles > 0;  // no MMA wrote the accumulator otherwise
+#pragma unroll
+      for (int c = 0; c < C::D; ++c) out[c] = any ? __uint_as_float(acc[c]) * sc : 0.f;
+      out[C::D] = !isE && p == 0 ? 1.f : 0.f;
+      part_c[(static_cast<size_t>(z) * P + p) * nsb + j] = 0.f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tbase, 64);
+}
+
+// ============================================================================
 // Query pass
 // ============================================================================
 // Where a query tile lies: query head bh (= b * H + h), 128-row tile qt within it, gq = bh % G and
@@ -1446,9 +1596,10 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   return FAVOR_OK;
 }
 
-// img: the state images of the plan's kv heads; W: m rows of d floats, w_row floats apart
+// img: the state images of the plan's kv heads; W: m rows of d floats, w_row floats apart (cpk > 0:
+// one W per kv head, w_head floats apart, and cpk CTAs per kv head)
 int launch_query_d64_img(const void* Q, const float* W, int w_row, float wscale, const unsigned char* img, void* out,
-                         const Plan& p, cudaStream_t st, bool overlap, bool relu) {
+                         const Plan& p, cudaStream_t st, bool overlap, bool relu, long w_head = 0, int cpk = 0) {
   using C = QueryD64;
   CUtensorMap mq, mo;
   const int bh = p.B * p.H;
@@ -1466,10 +1617,36 @@ int launch_query_d64_img(const void* Q, const float* W, int w_row, float wscale,
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass attribute: %s", cudaGetErrorString(e));
   const int ntiles = bh * ((p.L + 127) / 128);
-  const int grid = ntiles < num_sms() ? ntiles : num_sms();
+  const int grid = cpk > 0 ? p.B * p.Hkv * cpk : (ntiles < num_sms() ? ntiles : num_sms());
   e = launch_overlapped(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, overlap, mq, mo, W, img, p.L, p.m, p.H,
-                        p.Hkv, ntiles, static_cast<int>(p.op_bytes), wscale, w_row);
+                        p.Hkv, ntiles, static_cast<int>(p.op_bytes), wscale, w_row, w_head, cpk);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass launch: %s", cudaGetErrorString(e));
+  return FAVOR_OK;
+}
+
+// E, F: [kp][L] fp32; split: scratch of linformer_split_bytes; partials: the plan's (B = 2 B' batches)
+int launch_linformer_proj(const void* K, const void* V, const float* E, const float* F, void* split, void* partials,
+                          const Plan& pk, int heads, cudaStream_t st) {
+  using C = LinProj;
+  const int kpad = (pk.m + 127) / 128 * 128, Lpad = (pk.L + 63) / 64 * 64;
+  const int threads = 256, blocks = 4 * num_sms();
+  split_hi_lo_kernel<<<blocks, threads, 0, st>>>(E, F, static_cast<__nv_bfloat16*>(split), pk.m, kpad, pk.L, Lpad);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "projection split launch: %s", cudaGetErrorString(e));
+  CUtensorMap mef, mk, mv;
+  int rc = make_map(&mef, split, Lpad, kpad, 4);  // [4][kpad][Lpad]: boxes of 128 rows x 64 tokens
+  if (rc == FAVOR_OK) rc = make_map(&mk, K, C::D, pk.L, heads, C::TT);
+  if (rc == FAVOR_OK) rc = make_map(&mv, V, C::D, pk.L, heads, C::TT);
+  if (rc != FAVOR_OK) return rc;
+  e = cudaFuncSetAttribute(linformer_proj_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "projection attribute: %s", cudaGetErrorString(e));
+  char* base = static_cast<char*>(partials);
+  const float kscale = static_cast<float>(1.0 / std::sqrt(std::sqrt(static_cast<double>(C::D))));
+  e = launch_overlapped(linformer_proj_sm100, dim3(kpad / 128, pk.P, 2 * heads), dim3(C::THREADS), C::SMEM, st,
+                        false, mef, mk, mv, reinterpret_cast<float*>(base + pk.part_S_off),
+                        reinterpret_cast<float*>(base + pk.part_c_off), pk.L, pk.m, pk.P, pk.chunk, pk.nsb, heads,
+                        kscale);
+  if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "projection launch: %s", cudaGetErrorString(e));
   return FAVOR_OK;
 }
 
@@ -1494,27 +1671,27 @@ int sm100_key_pass(const void* K, const void* V, const float* W, void* partials,
                    : launch_key<128>(K, V, W, partials, p, st, overlap);
 }
 
+size_t linformer_split_bytes(int kp, int L) { return 4ull * ((kp + 127) / 128 * 128) * ((L + 63) / 64 * 64) * 2; }
+
+int sm100_linformer_proj(const void* K, const void* V, const float* E, const float* F, void* split, void* partials,
+                         const Plan& pk, int heads, cudaStream_t st) {
+  if (pk.d != 64) return set_error(FAVOR_ERR_UNSUPPORTED, "sm100 projection: needs d = 64");
+  if (pk.chunk % LinProj::TT != 0) return set_error(FAVOR_ERR_UNSUPPORTED, "sm100 projection: chunk not a whole number of stages");
+  return launch_linformer_proj(K, V, E, F, split, partials, pk, heads, st);
+}
+
 int sm100_linformer_query(const void* Q, const void* state, void* out, const Plan& pq, const Plan& pk, cudaStream_t st) {
   if (!(pq.d == 64 && pq.m > 64 && pq.m <= QueryD64::MMAX))
     return set_error(FAVOR_ERR_UNSUPPORTED, "sm100 projected query: needs d = 64 and 64 < k <= 512");
-  // one launch per kv head t: its G query heads (b H + h G .. + G - 1 = G t ..) are contiguous, its
-  // projected keys d^-1/4 E K are the state rows of head B Hkv + t (rows d + 1 floats apart) and F V
-  // is the state image of head t
-  const int heads = pq.B * pq.Hkv, G = pq.H / pq.Hkv, D1 = pq.d + 1;
-  Plan p1;
-  int rc = make_plan(1, G, 1, pq.L, pq.d, pq.m, &p1);
-  if (rc != FAVOR_OK) return rc;
+  // one launch: each kv head t gets its own CTAs (its W, the projected keys d^-1/4 E K, is the state
+  // rows of head B Hkv + t, rows d + 1 floats apart; its projected values F V are the state image of
+  // head t).  The CTAs read W before any wait, and W is the reduction's output: an ordinary launch.
+  const int heads = pq.B * pq.Hkv, D1 = pq.d + 1, G = pq.H / pq.Hkv, ntq = (pq.L + 127) / 128;
+  const int cpk = std::max(1, std::min(G * ntq, (num_sms() + heads / 2) / heads));
   const float* S = reinterpret_cast<const float*>(static_cast<const char*>(state) + pk.st_S_off);
   const unsigned char* img = static_cast<const unsigned char*>(state) + pk.st_op_off;
-  const size_t qstride = static_cast<size_t>(G) * pq.L * pq.d * 2;  // bytes of bf16 per kv head's queries
-  for (int t = 0; t < heads && rc == FAVOR_OK; ++t)
-    // the first launch reads the reduction's output before any wait: an ordinary launch; later ones
-    // follow query launches, which write only their own output rows
-    rc = launch_query_d64_img(static_cast<const char*>(Q) + t * qstride,
-                              S + (static_cast<size_t>(heads) + t) * pq.m * D1, D1, pq.wscale,
-                              img + static_cast<size_t>(t) * pk.op_bytes, static_cast<char*>(out) + t * qstride, p1, st,
-                              t > 0, false);
-  return rc;
+  return launch_query_d64_img(Q, S + static_cast<size_t>(heads) * pq.m * D1, D1, pq.wscale, img, out, pq, st, false,
+                              false, static_cast<long>(pq.m) * D1, cpk);
 }
 
 int sm100_query_pass_relu(const void* Q, const float* W, const void* state, void* out, const Plan& p, cudaStream_t st) {

@@ -75,7 +75,7 @@ template <bool RELU>
 __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, const float* __restrict__ W,
     const unsigned char* __restrict__ op_img, int L, int m, int H, int Hkv, int ntiles_total, int op_bytes,
-    float wscale, int w_row) {
+    float wscale, int w_row, long w_head, int cpk) {
   using C = QueryD64;
   constexpr int NQS = C::NQS;
   extern __shared__ unsigned char smem_raw[];
@@ -86,9 +86,20 @@ __global__ void __launch_bounds__(QueryD64::THREADS, 1) query_pass_d64_sm100(
   const int ntq = (L + 127) / 128;
   const int G = H / Hkv;
   const int nb = (m + C::FB - 1) / C::FB;  // blocks per tile (>= 2: m > 64)
-  const int per = ntiles_total / gridDim.x, extra = ntiles_total % gridDim.x;
-  const int T0 = blockIdx.x * per + min(static_cast<int>(blockIdx.x), extra);
-  const int n = per + (static_cast<int>(blockIdx.x) < extra ? 1 : 0);
+  // the CTA's tiles: an even share of all of them, or (cpk > 0: a W per kv head, w_head floats
+  // apart) an even share of one kv head's, so that the CTA's W is one kv head's throughout
+  int T0, n;
+  if (cpk > 0) {
+    const int hd = static_cast<int>(blockIdx.x) / cpk, c = static_cast<int>(blockIdx.x) % cpk, tph = G * ntq;
+    const int per = tph / cpk, extra = tph % cpk;
+    T0 = hd * tph + c * per + min(c, extra);
+    n = per + (c < extra ? 1 : 0);
+    W += static_cast<size_t>(hd) * w_head;
+  } else {
+    const int per = ntiles_total / gridDim.x, extra = ntiles_total % gridDim.x;
+    T0 = blockIdx.x * per + min(static_cast<int>(blockIdx.x), extra);
+    n = per + (static_cast<int>(blockIdx.x) < extra ? 1 : 0);
+  }
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
   int* img_count = reinterpret_cast<int*>(smem + C::S_IMGS);
   uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
