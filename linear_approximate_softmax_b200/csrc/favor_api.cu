@@ -264,14 +264,14 @@ int linformer_impl(int dtype, const void* Q, const void* K, const void* V, const
   Plan pq, pk;
   FAVOR_TRY(make_plan(B, H, Hkv, L, d, kp, &pq));
   FAVOR_TRY(make_plan(2 * B, H, Hkv, L, d, kp, &pk));  // the projected keys ride as B more batches
-  // bf16 with d = 64: the projections on the tensor cores, in enough key chunks for about six
-  // waves of CTAs (128 projected rows x chunk x product each)
+  // bf16 with d = 64: the projections on the tensor cores, in enough key chunks for about two
+  // waves of CTAs (128 projected rows x chunk x product x 4 kv heads each)
   const bool tc = dtype == FAVOR_BF16 && d == 64;
   if (tc) {
     int sms = 0;
     FAVOR_TRY(device_sm_count(&sms));
-    const long per_chunk = static_cast<long>((kp + 127) / 128) * 2 * B * Hkv;
-    plan_set_chunks(&pk, static_cast<int>(std::max(1L, (6L * sms + per_chunk - 1) / per_chunk)));
+    const long per_chunk = static_cast<long>((kp + 127) / 128) * 2 * ((B * Hkv + 3) / 4);
+    plan_set_chunks(&pk, static_cast<int>(std::max(1L, (2L * sms + per_chunk - 1) / per_chunk)));
   }
   keep_pool_mapped();
   void* ws = nullptr;

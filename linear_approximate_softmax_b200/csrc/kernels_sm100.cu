@@ -816,26 +816,29 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
 // Linformer projections on the tensor cores (d = 64, bf16 K and V)
 // ============================================================================
 // Linformer notes page, "4 Model": E K and F V (k x d per kv head).  E and F (fp32) are first
-// split into bf16 hi + lo (hi = bf16(x), lo = bf16(x - hi): about 16 bits of x).  One CTA takes a
-// (128 projected rows, key chunk, product) and accumulates (Ehi + Elo)[rows, chunk] K[chunk, :]
-// in tensor memory (M = 128, N = 64, 16 tokens per MMA; the E tile K-major, the K tile MN-major,
-// both as loaded), then writes the key pass's partial-state layout: F V with the constant column
-// 1 on chunk 0 only (the reduction's sum is then 1) as head h, d^-1/4 E K as head heads + h,
-// every stabiliser 0.
+// split into bf16 hi + lo (hi = bf16(x), lo = bf16(x - hi): about 16 bits of x).  One CTA takes
+// (128 projected rows, key chunk, product, group of HPC kv heads): E is shared by the kv heads, so
+// the K tiles of the group's heads sit side by side as one MN-major B operand (N = 64 HPC, one
+// 64-column group per head) and each E tile serves them all.  It accumulates (Ehi + Elo)[rows,
+// chunk] [K_h ...][chunk, :] in tensor memory (M = 128, 16 tokens per MMA), then writes the key
+// pass's partial-state layout: F V with the constant column 1 on chunk 0 only (the reduction's sum
+// is then 1) as head h, d^-1/4 E K as head heads + h, every stabiliser 0.
 struct LinProj {
   static constexpr int D = 64;
+  static constexpr int HPC = 4;  // kv heads per CTA
   // warp 0 TMA producer, warp 1 MMA issuer, warps 2-5 epilogue (TMEM lane quarter = warp % 4)
   static constexpr int THREADS = 192;
-  static constexpr int NST = 4;                  // stages of TT tokens
+  static constexpr int NST = 3;                  // stages of TT tokens
   static constexpr int TT = 64;
   static constexpr int A_TILE = 128 * TT * 2;    // 128 rows x 64 tokens, bf16, K-major SW128
-  static constexpr int B_TILE = TT * D * 2;      // 64 tokens x 64 dims, bf16, MN-major SW128
-  static constexpr int STAGE = 2 * A_TILE + B_TILE;  // E hi, E lo, K (or F hi, F lo, V)
+  static constexpr int B_TILE = TT * D * 2;      // one head: 64 tokens x 64 dims, bf16, MN-major SW128
+  static constexpr int STAGE = 2 * A_TILE + HPC * B_TILE;  // E hi, E lo, the heads' K (or F, V)
   static constexpr int S_BAR = NST * STAGE;
   static constexpr int B_FULL = 0, B_EMPTY = NST, B_DONE = 2 * NST, NBAR = 2 * NST + 1;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int SMEM = S_ABORT + 16 + 1024;
+  static constexpr int TCOLS = HPC * D;          // accumulator columns: 64 per head
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(A_TILE % 1024 == 0 && B_TILE % 1024 == 0, "swizzled operands on 1024-byte boundaries");
 };
@@ -868,9 +871,11 @@ __global__ void __launch_bounds__(LinProj::THREADS, 1) linformer_proj_sm100(
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int mt = blockIdx.x, p = blockIdx.y, z = blockIdx.z;
-  const bool isE = z >= heads;  // E K of kv head z - heads, or F V of kv head z
-  const int head = isE ? z - heads : z;
+  const int mt = blockIdx.x, p = blockIdx.y;
+  const int ngroups = (heads + C::HPC - 1) / C::HPC;
+  const bool isE = static_cast<int>(blockIdx.z) >= ngroups;  // E K or F V of a group of kv heads
+  const int h0 = (isE ? static_cast<int>(blockIdx.z) - ngroups : static_cast<int>(blockIdx.z)) * C::HPC;
+  const int nh = min(C::HPC, heads - h0);  // the group's kv heads (the last group may be short)
   const int t_begin = p * chunk, t_end = min(L, t_begin + chunk);
   const int ntiles = (t_end - t_begin + C::TT - 1) / C::TT;  // chunk is a multiple of TT: only L cuts a stage
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
@@ -892,7 +897,7 @@ __global__ void __launch_bounds__(LinProj::THREADS, 1) linformer_proj_sm100(
     prefetch_tmap(tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tptr_slot), 64);
+    tmem_alloc(smem_u32(tptr_slot), C::TCOLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -909,10 +914,12 @@ __global__ void __launch_bounds__(LinProj::THREADS, 1) linformer_proj_sm100(
         if (i >= C::NST && !mbar_wait<true>(bar(C::B_EMPTY + s), ((i / C::NST) - 1) & 1, abort_flag, err)) break;
         const int t0 = t_begin + C::TT * i;
         const uint32_t st = sbase + s * C::STAGE;
-        mbar_arrive_expect_tx(bar(C::B_FULL + s), C::STAGE);
+        // the columns of absent heads (a short last group) are left as they are: computed, never written
+        mbar_arrive_expect_tx(bar(C::B_FULL + s), 2 * C::A_TILE + nh * C::B_TILE);
         tma_load_3d(st, &tmEF, bar(C::B_FULL + s), t0, 128 * mt, zs);  // x = token, y = row, z = split
         tma_load_3d(st + C::A_TILE, &tmEF, bar(C::B_FULL + s), t0, 128 * mt, zs + 1);
-        tma_load_3d(st + 2 * C::A_TILE, tmB, bar(C::B_FULL + s), 0, t0, head);  // x = dim, y = token, z = head
+        for (int n = 0; n < nh; ++n)  // x = dim, y = token, z = kv head
+          tma_load_3d(st + 2 * C::A_TILE + n * C::B_TILE, tmB, bar(C::B_FULL + s), 0, t0, h0 + n);
         issued = i + 1;
       }
       for (int i = max(0, issued - C::NST); i < issued; ++i)  // no copy is in flight when the CTA leaves
@@ -920,7 +927,7 @@ __global__ void __launch_bounds__(LinProj::THREADS, 1) linformer_proj_sm100(
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---------------- MMA issuer ----------------
-      const uint32_t idesc = idesc_bf16(128, C::D, false, true);
+      const uint32_t idesc = idesc_bf16(128, C::TCOLS, false, true);
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % C::NST;
         if (!mbar_wait(bar(C::B_FULL + s), (i / C::NST) & 1, abort_flag, err)) break;
@@ -928,7 +935,8 @@ __global__ void __launch_bounds__(LinProj::THREADS, 1) linformer_proj_sm100(
         const uint32_t st = sbase + s * C::STAGE;
 #pragma unroll
         for (int kk = 0; kk < C::TT / 16; ++kk) {  // 16 tokens per step: Ehi then Elo against the same K rows
-          const uint64_t bd = sdesc_sw128(st + 2 * C::A_TILE + 2048 * kk, 16, 1024);
+          // B: the heads' 64-column groups B_TILE bytes apart (LBO), 8-token groups 1024 apart (SBO)
+          const uint64_t bd = sdesc_sw128(st + 2 * C::A_TILE + 2048 * kk, C::B_TILE, 1024);
           mma_ss(tbase, sdesc_sw128(st + 32 * kk, 16, 1024), bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
           mma_ss(tbase, sdesc_sw128(st + C::A_TILE + 32 * kk, 16, 1024), bd, idesc, 1u);
         }
@@ -936,30 +944,33 @@ __global__ void __launch_bounds__(LinProj::THREADS, 1) linformer_proj_sm100(
       }
       mma_commit(bar(C::B_DONE));  // arrives once every MMA above has completed
     }
-  } else {  // ---------------- epilogue: one projected row per thread ----------------
+  } else {  // ---------------- epilogue: one projected row per thread, for each head of the group ----------------
     const int eq = warp & 3;
     const int r = eq * 32 + lane, j = 128 * mt + r;
     const bool ok = mbar_wait(bar(C::B_DONE), 0, abort_flag, err, 200000000ull);
     tc_fence_after();
-    uint32_t acc[64];
-    tmem_ld32(taddr(tbase, eq, 0), *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
-    tmem_ld32(taddr(tbase, eq, 32), *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
-    tmem_wait_ld();
-    if (j < kp) {
-      float* out = part_S + (static_cast<size_t>(z) * P + p) * static_cast<size_t>(kp) * (C::D + 1) +
-                   static_cast<size_t>(j) * (C::D + 1);
-      const float sc = isE ? kscale : 1.f;
-      const bool any = ok && ntiles > 0;  // no MMA wrote the accumulator otherwise
+    const float sc = isE ? kscale : 1.f;
+    const bool any = ok && ntiles > 0;  // no MMA wrote the accumulator otherwise
+    for (int n = 0; n < nh; ++n) {
+      uint32_t acc[64];
+      tmem_ld32(taddr(tbase, eq, 64 * n), *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
+      tmem_ld32(taddr(tbase, eq, 64 * n + 32), *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
+      tmem_wait_ld();
+      if (j < kp) {
+        const int z = (isE ? heads : 0) + h0 + n;  // F V as head h, E K as head heads + h
+        float* out = part_S + (static_cast<size_t>(z) * P + p) * static_cast<size_t>(kp) * (C::D + 1) +
+                     static_cast<size_t>(j) * (C::D + 1);
 #pragma unroll
-      for (int c = 0; c < C::D; ++c) out[c] = any ? __uint_as_float(acc[c]) * sc : 0.f;
-      out[C::D] = !isE && p == 0 ? 1.f : 0.f;
-      part_c[(static_cast<size_t>(z) * P + p) * nsb + j] = 0.f;
+        for (int c = 0; c < C::D; ++c) out[c] = any ? __uint_as_float(acc[c]) * sc : 0.f;
+        out[C::D] = !isE && p == 0 ? 1.f : 0.f;
+        part_c[(static_cast<size_t>(z) * P + p) * nsb + j] = 0.f;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tbase, 64);
+  if (warp == 1) tmem_dealloc(tbase, C::TCOLS);
 }
 
 // ============================================================================
@@ -1642,7 +1653,8 @@ int launch_linformer_proj(const void* K, const void* V, const float* E, const fl
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "projection attribute: %s", cudaGetErrorString(e));
   char* base = static_cast<char*>(partials);
   const float kscale = static_cast<float>(1.0 / std::sqrt(std::sqrt(static_cast<double>(C::D))));
-  e = launch_overlapped(linformer_proj_sm100, dim3(kpad / 128, pk.P, 2 * heads), dim3(C::THREADS), C::SMEM, st,
+  e = launch_overlapped(linformer_proj_sm100, dim3(kpad / 128, pk.P, 2 * ((heads + C::HPC - 1) / C::HPC)),
+                        dim3(C::THREADS), C::SMEM, st,
                         false, mef, mk, mv, reinterpret_cast<float*>(base + pk.part_S_off),
                         reinterpret_cast<float*>(base + pk.part_c_off), pk.L, pk.m, pk.P, pk.chunk, pk.nsb, heads,
                         kscale);
