@@ -198,22 +198,37 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
   const bool live = f < m;
   const float* pc = part_c + static_cast<size_t>(head) * P * nsb;
   const float* rows = part_S + (static_cast<size_t>(head) * P * m + f) * D1;  // chunk p at + p * m * D1
-  float x[CB][NC];
-  auto load = [&](int p0) {
+  float x[CB][NC], cc[CB];
+  auto load = [&](int p0) {  // CB chunks' rows of this feature and their stabilisers, all in flight at once
 #pragma unroll
-    for (int b = 0; b < CB; ++b)
+    for (int b = 0; b < CB; ++b) {
+      cc[b] = live && p0 + b < P ? pc[(p0 + b) * nsb + f / kStabBlock] : -INFINITY;
 #pragma unroll
       for (int k = 0; k < NC; ++k) {
         const int n = g + 8 * k;
         x[b][k] = live && p0 + b < P && n < D1 ? rows[static_cast<size_t>(p0 + b) * m * D1 + n] : 0.f;
       }
+    }
   };
   load(0);
+  // the stabiliser maxima, eight independent loads in flight at a time
   float cf = -INFINITY;  // this feature's largest chunk stabiliser
   if (live)
-    for (int p = 0; p < P; ++p) cf = fmaxf(cf, pc[p * nsb + f / kStabBlock]);
+    for (int p0 = 0; p0 < P; p0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = p0 + u < P ? pc[(p0 + u) * nsb + f / kStabBlock] : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) cf = fmaxf(cf, v[u]);
+    }
   float cs = -INFINITY;  // the head's largest stabiliser
-  for (int i = tid; i < P * nsb; i += kThreads) cs = fmaxf(cs, pc[i]);
+  for (int i0 = tid; i0 < P * nsb; i0 += 8 * kThreads) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = i0 + u * kThreads < P * nsb ? pc[i0 + u * kThreads] : -INFINITY;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) cs = fmaxf(cs, v[u]);
+  }
   float val[NC];
 #pragma unroll
   for (int k = 0; k < NC; ++k) val[k] = 0.f;
@@ -223,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
     for (int b = 0; b < CB; ++b) {
       const int p = p0 + b;
       if (live && p < P) {
-        const float c = pc[p * nsb + f / kStabBlock];
+        const float c = cc[b];
         const float w = c == -INFINITY ? 0.f : exp2f(c - cf);
 #pragma unroll
         for (int k = 0; k < NC; ++k) val[k] = fmaf(w, x[b][k], val[k]);
