@@ -77,8 +77,8 @@ def load_peaks():
 # from one ncu capture of the kernel as it stands; an entry is removed whenever its kernel changes
 # (the bench then reports traffic null until the kernel is captured again).
 PROFILED_TRAFFIC = {
-    # query_pass_d64_sm100 as of "issue the next projection right after the contraction ..."
-    ("bf16_L16384_heavykeys", "query_pass"): 157.59e6,
+    # query_pass_d64_sm100<false> as of "Linformer on the tensor cores end to end ..." (W row stride, per-head W)
+    ("bf16_L16384_heavykeys", "query_pass"): 157.76e6,
     # key_pass_pp_sm100 as of "256 features per key-pass CTA, key norms in their own warp ..."
     ("bf16_L16384_heavykeys", "key_pass"): 205.87e6,
 }
