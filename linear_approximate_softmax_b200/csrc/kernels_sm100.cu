@@ -1004,16 +1004,17 @@ struct TileCursor {
 
 template <int D>
 struct QueryCfg {
-  // warp 0 TMA producer, warps 1-2 MMA issuers (one per warpgroup), warp 3 idle,
+  // warp 0 TMA producer, warps 1-2 MMA issuers (one per warpgroup), warp 3 state images,
   // warps 4-11 two epilogue warpgroups on alternate tiles
   static constexpr int THREADS = 384;
   static constexpr int EPI0 = 4;
-  static constexpr int FB = D == 64 ? 128 : 64;      // features per block (MMA1 N, MMA2 K)
+  static constexpr int FB = 128;                     // features per block (MMA1 N, MMA2 K)
   static constexpr int MMAX = D == 64 ? 512 : 256;   // features held in shared memory
   static constexpr int QTILE = 128 * D * 2;
   static constexpr int SP = D * 128 * (MMAX / 64) + 8 * MMAX;  // fp16 image, exponents, fp32 normaliser column
-  // TMEM columns: warpgroup w owns U at w * TSTRIDE, then phi' (FB / 2 columns of fp16 pairs), then O
-  static constexpr int TSTRIDE = FB + FB / 2 + D;
+  // TMEM columns: warpgroup w owns U at w * TSTRIDE (phi' as fp16 pairs over its first FB / 2
+  // columns once U is read), then O
+  static constexpr int TSTRIDE = FB + D;
   static_assert(2 * TSTRIDE <= 512, "TMEM budget");
   // shared memory
   static constexpr int S_W = 0;                          // W' fp16, [D/64 regions][MMAX rows][128 B]
@@ -1026,8 +1027,8 @@ struct QueryCfg {
   static constexpr int NSLOT = OWN_SLOT ? 8 : 4;
   static constexpr int S_STG = S_Q + 2 * QTILE;
   static constexpr int S_BAR = S_STG + NSLOT * 32 * 128;
-  static constexpr int B_QF = 0, B_QE = 2, B_CVT = 4, B_UF = 6, B_UE = 8, B_PHI = 10, B_M2 = 12, B_OF = 14,
-                       B_OE = 16, B_SF = 18, B_SE = 19, B_STG = 20, NBAR = 24;
+  static constexpr int B_QF = 0, B_QE = 2, B_CVT = 4, B_UF = 6, B_PHI = 8, B_M2 = 10, B_OF = 12, B_OE = 14,
+                       B_SF = 16, B_SE = 17, B_STG = 18, NBAR = 22;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int S_IMGS = S_ABORT + 4;  // state images loaded so far (published by warp 3)
@@ -1037,16 +1038,18 @@ struct QueryCfg {
 };
 
 // Query pass.  The CTA's tiles go alternately to two epilogue warpgroups, each with its own
-// U, phi' and O buffers in tensor memory, its own Q stage and its own MMA-issuing thread, so
-// one warpgroup's exponentials overlap the other's tensor-memory reads, waits and output.
-// Per block of FB features a warpgroup reads U twice: once for the exact row max of
-// 2^k U + e, once to exponentiate; as soon as the second read is done U is released, so the
-// next block's projection runs while this block's exponentials and contraction finish.  The
-// row stabiliser is raised lazily across blocks with an exact rescale of O and of the
-// normaliser, which the epilogue sums itself (phi' times the state's fp32 normaliser
-// column).  The projection runs in fp16: each warpgroup rewrites its next Q tile in place as
-// fp16 times 2^-k, one k per row that puts the row's largest |q| in [2^14, 2^15), and
-// multiplies that row's U by 2^k.
+// U and O buffers in tensor memory, its own Q stage and its own MMA-issuing thread, so one
+// warpgroup's exponentials run while the tensor cores serve the other's contraction and next
+// projection.  Blocks are 128 features wide (at d = 128 a 128-wide projection costs the tensor
+// pipe as many cycles per MMA as a 64-wide one, so the wider block halves the projection MMAs);
+// phi' goes as fp16 pairs over the first half of the block's own U columns, and the next
+// projection is issued right behind the contraction that reads them (one thread's MMAs execute
+// in issue order), so U's arrival also means the previous contraction has completed.  The row
+// stabiliser is raised lazily across blocks with an exact rescale of O and of the normaliser,
+// which the epilogue sums itself (phi' times the state's fp32 normaliser column).  The
+// projection runs in fp16: each warpgroup rewrites its next Q tile in place as fp16 times 2^-k,
+// one k per row that puts the row's largest |q| in [2^14, 2^15), and multiplies that row's U by
+// 2^k.
 template <int D>
 __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO, const float* __restrict__ W,
@@ -1083,9 +1086,8 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       mbar_init(bar(C::B_QE + i), 1);
       mbar_init(bar(C::B_CVT + i), 4);  // one arrival per epilogue warp
       mbar_init(bar(C::B_UF + i), 1);
-      mbar_init(bar(C::B_UE + i), 4);
       mbar_init(bar(C::B_PHI + i), 4);
-      mbar_init(bar(C::B_M2 + i), 1);
+      mbar_init(bar(C::B_M2 + i), 1);   // the issuer's final drain
       mbar_init(bar(C::B_OF + i), 1);
       mbar_init(bar(C::B_OE + i), 4);
     }
@@ -1194,13 +1196,14 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     }
   } else if (warp == 1 || warp == 2) {
     // ---------------- MMA issuer of warpgroup w = warp - 1: its tiles w, w + 2, ... ----------------
-    // Within a tile the next block's projection goes out as soon as the epilogue has read this
-    // block's U, ahead of this block's contraction; across tiles it waits for the next tile's
-    // Q, which the epilogue converts after handing over the tile's last block.
+    // Per block: the contraction once phi' is stored (and, on a tile's first block, O read out),
+    // then at once the next block's projection into the same columns; across tiles that
+    // projection waits for the next tile's Q, which the epilogue converts after handing over the
+    // tile's last block.
     if (lane == 0) {
       const int w = warp - 1;
       const uint32_t id2 = idesc_f16(128, D, false, false);
-      const uint32_t dU = tbase + w * C::TSTRIDE, dP = dU + FB, dO = dP + FB / 2;
+      const uint32_t dU = tbase + w * C::TSTRIDE, dO = dU + FB;
       const uint32_t qbase = sbase + C::S_Q + w * C::QTILE;
       const int ntw = (n - w + 1) / 2;  // my tiles
       const int nblk = ntw * nb;        // my blocks
@@ -1215,7 +1218,8 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         return true;
       };
       // U = (2^-k Q) W'^T in fp16 for my block b, always FB columns wide: W' rows past m are
-      // zero, so every U column the epilogue reads is written (its e = -inf masks it)
+      // zero, so every U column the epilogue reads is written (its e = -inf masks it).  The
+      // commit also covers the contraction issued before it.
       const uint32_t id1 = idesc_f16(128, FB, false, false);
       auto mma1 = [&](int j) {
 #pragma unroll
@@ -1247,11 +1251,6 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       for (int b = 0, tc = 0, j = 0; b < nblk && ok; ++b) {
         const int t = w + 2 * tc, k = cur.img;
         const bool more = b + 1 < nblk, boundary = (j == nb - 1);
-        if (more && !boundary) {  // next block of the same tile
-          if (!mbar_wait(bar(C::B_UE + w), b & 1, abort_flag, err)) break;
-          tc_fence_after();
-          mma1(j + 1);
-        }
         if (!mbar_wait(bar(C::B_PHI + w), b & 1, abort_flag, err)) break;
         if (j == 0) {
           if (tc >= 1 && !mbar_wait(bar(C::B_OE + w), (tc - 1) & 1, abort_flag, err)) break;
@@ -1262,9 +1261,8 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
         for (int ks = 0; ks < bw / 16; ++ks) {  // MMA2: O += phi' S', 16 features per step, two per TMEM column
           const int fk = FB * j + 16 * ks;
           const uint64_t bd = sdesc_sw128(sbase + C::S_SP + (fk >> 6) * (D * 128) + 32 * ((fk & 63) >> 4), 16, 1024);
-          mma_ts(dO, dP + 8 * ks, bd, id2, (j > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(dO, dU + 8 * ks, bd, id2, (j > 0 || ks > 0) ? 1u : 0u);
         }
-        mma_commit(bar(C::B_M2 + w));
         if (boundary) {
           mma_commit(bar(C::B_OF + w));
           TileCursor nx = cur;  // my next tile, t + 2
@@ -1274,8 +1272,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
             mma_commit(bar(C::B_SE));
             rel = k + 1;
           }
-          if (more) {  // first block of my next tile: U read and that tile's Q converted
-            if (!mbar_wait(bar(C::B_UE + w), b & 1, abort_flag, err)) break;
+          if (more) {  // first block of my next tile, once its Q is converted
             if (!enter_tile(tc + 1, nx.img)) break;
             tc_fence_after();
             mma1(0);
@@ -1284,11 +1281,15 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
           ++tc;
           j = 0;
         } else {
+          mma1(j + 1);  // behind the contraction that reads phi' from the same columns
           ++j;
         }
       }
       while (ok && rel < nimg - 1) ok = release_unused();
-      if (nblk >= 1) mbar_wait(bar(C::B_M2 + w), (nblk - 1) & 1, abort_flag, err, 200000000ull);
+      if (nblk >= 1) {  // everything I issued has completed
+        mma_commit(bar(C::B_M2 + w));
+        mbar_wait(bar(C::B_M2 + w), 0, abort_flag, err, 200000000ull);
+      }
     }
   }
   } else {
@@ -1297,7 +1298,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     const int eq = warp & 3;
     const int ewg = (warp - C::EPI0) >> 2;
     const int r = eq * 32 + lane;  // query row within the tile (TMEM lane)
-    const uint32_t cU = ewg * C::TSTRIDE, cP = cU + FB, cO = cP + FB / 2;  // TMEM columns
+    const uint32_t cU = ewg * C::TSTRIDE, cO = cU + FB;  // TMEM columns: U, then phi' over it; O
     // the image holds [atoms][D rows][64 features] fp16, then e and the normaliser column (fp32,
     // same scaling as the image), each over m rounded up to 128 features, e = -inf past m
     const int atoms = (m + 63) / 64, tail = (m + 127) / 128 * 128;
@@ -1357,16 +1358,13 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       wait_count_above(img_count, ec.img, abort_flag, err);  // this tile's image (exponents) is in
       float c = 0.f, den = 0.f;
       for (int j = 0; j < nb; ++j, ++cntb) {
+        // U of this block; its arrival also means the previous block's contraction has completed
         mbar_wait(bar(C::B_UF + ewg), cntb & 1, abort_flag, err);
         tc_fence_after();
-        // the whole block of this row into registers: one read of U, which is then released
         float v[FB];
 #pragma unroll
         for (int q4 = 0; q4 < FB / 32; ++q4) tmem_ld32(taddr(tbase, eq, cU + 32 * q4), *reinterpret_cast<uint32_t(*)[32]>(&v[32 * q4]));
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::B_UE + ewg));  // the next projection may overwrite U
         const float4* e4p = reinterpret_cast<const float4*>(ev + FB * j);
         const float4* s4p = reinterpret_cast<const float4*>(sd + FB * j);
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -1384,9 +1382,6 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
           m4[k4 & 3] = max3(m4[k4 & 3], v[4 * k4 + 2], v[4 * k4 + 3]);
         }
         const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        // the previous block's contraction must be complete before phi' is overwritten or O rescaled
-        if (cntb >= 1) mbar_wait(bar(C::B_M2 + ewg), (cntb - 1) & 1, abort_flag, err);
-        tc_fence_after();
         const bool need = (j > 0) && (mx > c + kTau);
         if (j == 0) c = mx;
         if (__any_sync(0xffffffffu, need)) {  // raise the stabiliser of the rows that need it
@@ -1395,9 +1390,9 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
           den *= f;
         }
         if (need) c = mx;
-        // phi' = 2^(2^k U + e - c) as fp16 pairs into the phi' buffer; normaliser in fp32
+        // phi' = 2^(2^k U + e - c) as fp16 pairs over U's first columns; normaliser in fp32
         const float2 nc2 = make_float2(-c, -c);
-        float2 den2 = make_float2(0.f, 0.f), den2b = make_float2(0.f, 0.f);  // two independent chains
+        float2 den2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int q4 = 0; q4 < FB / 32; ++q4) {
           uint32_t ph[16];
@@ -1408,13 +1403,13 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
             const float2 b01 = __fadd2_rn(make_float2(a[0], a[1]), nc2), b23 = __fadd2_rn(make_float2(a[2], a[3]), nc2);
             const float2 p01 = make_float2(ex2(b01.x), ex2(b01.y)), p23 = make_float2(ex2(b23.x), ex2(b23.y));
             den2 = __ffma2_rn(p01, make_float2(s4.x, s4.y), den2);
-            den2b = __ffma2_rn(p23, make_float2(s4.z, s4.w), den2b);
+            den2 = __ffma2_rn(p23, make_float2(s4.z, s4.w), den2);
             ph[2 * k4] = pack_f16x2(p01.x, p01.y);
             ph[2 * k4 + 1] = pack_f16x2(p23.x, p23.y);
           }
-          tmem_st16(taddr(tbase, eq, cP + 16 * q4), ph);
+          tmem_st16(taddr(tbase, eq, cU + 16 * q4), ph);
         }
-        den += (den2.x + den2.y) + (den2b.x + den2b.y);
+        den += den2.x + den2.y;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
