@@ -358,17 +358,24 @@ __global__ void __launch_bounds__(kThreads) query_pass_kernel(
       for (int f = k; f < m; f += 8) U[r * mp + f] = fmaxf(U[r * mp + f], 0.f);
     }
   }
-  __syncthreads();
   float acc[NE];
 #pragma unroll
   for (int k = 0; k < NE; ++k) acc[k] = 0.f;
-  for (int f = 0; f < m; ++f) {
+  // out rows += phi S, 64 state rows at a time staged in shared memory (in place of W'), the
+  // features summed in order f = 0 .. m - 1
+  for (int f0 = 0; f0 < m; f0 += kFB) {
+    const int fbw = min(kFB, m - f0);
+    __syncthreads();  // phi is in place / the previous rows are used
+    for (int i = tid; i < fbw * D1; i += kThreads) Ws[i] = Sh[static_cast<size_t>(f0) * D1 + i];
+    __syncthreads();
+    for (int f = 0; f < fbw; ++f) {
 #pragma unroll
-    for (int k = 0; k < NE; ++k) {
-      const int e = tid + k * kThreads;
-      if (e < kQT * D1) {
-        const int r = e / D1, c = e % D1;
-        acc[k] = fmaf(U[r * mp + f], Sh[static_cast<size_t>(f) * D1 + c], acc[k]);
+      for (int k = 0; k < NE; ++k) {
+        const int e = tid + k * kThreads;
+        if (e < kQT * D1) {
+          const int r = e / D1, c = e % D1;
+          acc[k] = fmaf(U[r * mp + f0 + f], Ws[f * D1 + c], acc[k]);
+        }
       }
     }
   }
