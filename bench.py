@@ -79,8 +79,8 @@ def load_peaks():
 PROFILED_TRAFFIC = {
     # query_pass_d64_sm100<false> as of "Linformer on the tensor cores end to end ..." (W row stride, per-head W)
     ("bf16_L16384_heavykeys", "query_pass"): 157.76e6,
-    # key_pass_pp_sm100 as of "256 features per key-pass CTA, key norms in their own warp ..."
-    ("bf16_L16384_heavykeys", "key_pass"): 205.87e6,
+    # key_pass_pp_sm100<true, false> as of "Key pass: the key norms folded into the projection ..."
+    ("bf16_L16384_heavykeys", "key_pass"): 205.39e6,
 }
 
 # Per-SM issue rates of one B200 SM per clock, times 148 SMs and the maximum SM clock: the MUFU

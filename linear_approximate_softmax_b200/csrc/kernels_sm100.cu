@@ -437,8 +437,12 @@ struct KeyPP {
   static constexpr int S_WHI = 0, S_WLO = NFEAT * 128;
   static constexpr int S_K = S_WLO + NFEAT * 128;
   static constexpr int S_V = S_K + NST * TILE;
-  static constexpr int S_NRM = S_V + NST * TILE;    // per stage: -n(k) [128]
-  static constexpr int S_CW = S_NRM + NST * 512;    // final stabilisers and normalisers, [2][2][128]
+  // per stage: n(k) of the tile's 128 tokens as bf16 hi, mid, lo (then 13 zeros), K-major with the
+  // 32-byte swizzle: the B operand of one more projection step against S_NA, whose rows are
+  // (-1, -1, -1, 0, ...), so that U^T comes out of the tensor core as W'k - n(k)
+  static constexpr int S_NB = S_V + NST * TILE;
+  static constexpr int S_NA = S_NB + NST * 4096;
+  static constexpr int S_CW = S_NA + 4096;          // final stabilisers and normalisers, [2][2][128]
   static constexpr int S_BAR = S_CW + 2048;
   // PHI and SDONE come in halves per warpgroup (2 w + h): the weights of tokens 64 h .. 64 h + 63
   // and the contraction steps that read them
@@ -474,7 +478,6 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
   constexpr int TSTEP = WIDE ? 1 : 2;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::S_ABORT);
   uint32_t* tptr_slot = reinterpret_cast<uint32_t*>(smem + C::S_TPTR);
-  float* nrm = reinterpret_cast<float*>(smem + C::S_NRM);
   float* cw = reinterpret_cast<float*>(smem + C::S_CW);
   auto bar = [&](int i) { return sbase + C::S_BAR + 8u * i; };
 
@@ -528,6 +531,17 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
     *reinterpret_cast<uint4*>(smem + C::S_WHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(smem + C::S_WLO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
+  // the norm step's A operand (row r, 16-byte chunk c at c ^ (r / 4 % 2)) and its B operands' zero
+  // chunks (the norm warp writes chunk 0 of each row per tile)
+  for (int r = tid; r < 128; r += C::THREADS) {
+    const int sw = (r >> 2) & 1;
+    *reinterpret_cast<uint4*>(smem + C::S_NA + r * 32 + (sw << 4)) = make_uint4(0xBF80BF80u, 0x0000BF80u, 0u, 0u);
+    *reinterpret_cast<uint4*>(smem + C::S_NA + r * 32 + ((1 ^ sw) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  for (int i = tid; i < C::NST * 128; i += C::THREADS) {
+    const int r = i & 127;
+    *reinterpret_cast<uint4*>(smem + C::S_NB + (i >> 7) * 4096 + r * 32 + ((1 ^ ((r >> 2) & 1)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -567,7 +581,7 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
       const uint32_t dU = tbase + w * C::T_STRIDE + C::T_U, dP = tbase + w * C::T_STRIDE + C::T_P,
                      dS = tbase + w * C::T_STRIDE + C::T_S;
       const uint32_t wrow = WIDE ? w * 128 * 128 : 0;  // this warpgroup's rows of W'
-      auto mma1 = [&](int i) {  // U^T = (W'hi + W'lo) K^T
+      auto mma1 = [&](int i) {  // U^T = (W'hi + W'lo) K^T (- n(k), once the tile's norms are in)
         const int s = i % C::NST;
 #pragma unroll
         for (int ks = 0; ks < 2 * (D / 16); ++ks) {
@@ -575,14 +589,20 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
           mma_ss(dU, sdesc_sw128(sbase + (ks < D / 16 ? C::S_WHI : C::S_WLO) + wrow + 32 * kk, 16, 1024),
                  sdesc_sw128(sbase + C::S_K + s * C::TILE + 32 * kk, 16, 1024), id1, ks > 0 ? 1u : 0u);
         }
+        if constexpr (!RELU) {
+          if (!mbar_wait(bar(C::B_NRM + s), (i / C::NST) & 1, abort_flag, err)) return false;
+          tc_fence_after();
+          mma_ss(dU, sdesc_sw32(sbase + C::S_NA, 256), sdesc_sw32(sbase + C::S_NB + s * 4096, 256), id1, 1u);
+        }
         mma_commit(bar(C::B_D1F + w));
+        return true;
       };
       int cnt = 0;
       const int first = WIDE ? 0 : w;
       bool ok = first < ntiles && mbar_wait(bar(C::B_KVF + first % C::NST), (first / C::NST) & 1, abort_flag, err);
       if (ok) {
         tc_fence_after();
-        mma1(first);
+        ok = mma1(first);
       }
       for (int i = first; i < ntiles && ok; i += TSTEP, ++cnt) {
         const int s = i % C::NST;
@@ -591,7 +611,7 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
           const int s2 = (i + TSTEP) % C::NST;
           if (!mbar_wait(bar(C::B_KVF + s2), ((i + TSTEP) / C::NST) & 1, abort_flag, err)) break;  // the next tile landed
           tc_fence_after();
-          mma1(i + TSTEP);
+          if (!mma1(i + TSTEP)) break;
         }
         // MMA2: S_w += phi^T V, 16 tokens per step, each half of the tile as soon as its weights are in
         for (int h = 0; h < 2 && ok; ++h) {
@@ -640,9 +660,20 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
         }
         const float sa = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
         const float sb = (acc[2].x + acc[2].y) + (acc[3].x + acc[3].y);
-        nrm[s * 128 + ta] = (t_begin + 128 * i + ta < t_end) ? -sa * nscale : -INFINITY;
-        nrm[s * 128 + tb] = (t_begin + 128 * i + tb < t_end) ? -sb * nscale : -INFINITY;
+        // n(k) as bf16 hi + mid + lo (exact residuals, ~24 bits); a token past the chunk end gets
+        // n = 2^100, which sends its exponent to -2^100 and its weight to 0
+        auto put = [&](int t, float nk) {
+          const uint32_t h = pack_bf16x2(nk, 0.f);
+          const float r1 = nk - __uint_as_float(h << 16);
+          const uint32_t hm = pack_bf16x2(nk, r1);
+          const float r2 = r1 - __uint_as_float(hm & 0xFFFF0000u);
+          *reinterpret_cast<uint4*>(smem + C::S_NB + s * 4096 + t * 32 + (((t >> 2) & 1) << 4)) =
+              make_uint4(hm, pack_bf16x2(r2, 0.f), 0u, 0u);
+        };
+        put(ta, (t_begin + 128 * i + ta < t_end) ? sa * nscale : 0x1p100f);
+        put(tb, (t_begin + 128 * i + tb < t_end) ? sb * nscale : 0x1p100f);
       }
+      fence_proxy_async_smem();  // the norms are read by the tensor cores
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::B_NRM + s));  // release: the 128 norms are stored
     }
@@ -684,7 +715,6 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
       mbar_wait(bar(C::B_D1F + ewg), cnt & 1, abort_flag, err);
       // the norms of tile i (the norm warp cannot have moved on to the stage's next tile: that
       // tile is loaded only after this one has been contracted)
-      if (!RELU) mbar_wait(bar(C::B_NRM + s), (i / C::NST) & 1, abort_flag, err);
       // this tile's U^T row into registers (one read), then release it to the next projection
       float ut[128];
 #pragma unroll
@@ -708,7 +738,6 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
       const float2 ncc = make_float2(-c_run, -c_run);
       float2 zs2 = make_float2(0.f, 0.f);
       float tm4[4] = {tmax, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
-      const float4* nv = reinterpret_cast<const float4*>(nrm + s * 128);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         if ((q4 & 1) == 0) {  // a new half: its phi columns are free once the previous tile's
@@ -725,9 +754,7 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
             p01 = make_float2(fmaxf(r[0], 0.f), fmaxf(r[1], 0.f));
             p23 = make_float2(fmaxf(r[2], 0.f), fmaxf(r[3], 0.f));
           } else {
-            const float4 n4 = nv[8 * q4 + k4];
-            const float2 a01 = __fadd2_rn(make_float2(r[0], r[1]), make_float2(n4.x, n4.y));
-            const float2 a23 = __fadd2_rn(make_float2(r[2], r[3]), make_float2(n4.z, n4.w));
+            const float2 a01 = make_float2(r[0], r[1]), a23 = make_float2(r[2], r[3]);  // W'k - n(k)
             tm4[k4 & 3] = max3(tm4[k4 & 3], a01.x, a01.y);
             tm4[k4 & 3] = max3(tm4[k4 & 3], a23.x, a23.y);
             const float2 b01 = __fadd2_rn(a01, ncc), b23 = __fadd2_rn(a23, ncc);

@@ -243,6 +243,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// K-major, 32-byte swizzle (rows of 16 bf16; 16-byte chunk c of row r at c ^ (r / 4 % 2)); SBO
+// = the stride of 8-row groups; the leading offset is unused for K-major swizzled layouts
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) |
+         (1ull << 46) | (6ull << 61);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]   (kind::f16: bf16 operands)
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
