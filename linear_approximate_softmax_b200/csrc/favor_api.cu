@@ -97,9 +97,12 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
   const int tiles = (L + kTileTokens - 1) / kTileTokens;
   // Key chunks: the tensor-core key pass runs one CTA per SM for each (kv head,
   // feature group, chunk).  Pick the chunk count that minimises the
-  // makespan in waves of CTAs, counting half a tile of start-up per wave.
+  // makespan in waves of CTAs, counting half a tile of start-up per wave, plus the
+  // partial state the chunks write and the reduction reads back (about 4 MB in the
+  // time a CTA spends on one key tile).
   const int nfeat = key_features_per_cta(d, m);
   const long units = static_cast<long>(heads) * ((m + nfeat - 1) / nfeat);
+  constexpr double kPartBytesPerTile = 4.0e6;
   double best = 1e300;
   int best_ct = tiles;
   for (int P = 1; P <= tiles; ++P) {
@@ -107,7 +110,8 @@ int make_plan(int B, int H, int Hkv, int L, int d, int m, Plan* p) {
     const long Pe = (tiles + ct - 1) / ct;
     if (Pe != P) continue;
     const long waves = (units * Pe + sms - 1) / sms;
-    const double cost = static_cast<double>(waves) * (ct + 0.5);
+    const double part_bytes = static_cast<double>(heads) * Pe * m * (d + 1) * sizeof(float);
+    const double cost = static_cast<double>(waves) * (ct + 0.5) + part_bytes / kPartBytesPerTile;
     if (cost < best - 1e-9) { best = cost; best_ct = ct; }
   }
   p->chunk = best_ct * kTileTokens;

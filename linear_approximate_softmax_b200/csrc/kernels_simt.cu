@@ -221,13 +221,18 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
 #pragma unroll
       for (int u = 0; u < 8; ++u) cf = fmaxf(cf, v[u]);
     }
-  float cs = -INFINITY;  // the head's largest stabiliser
-  for (int i0 = tid; i0 < P * nsb; i0 += 8 * kThreads) {
-    float v[8];
+  float cs = -INFINITY;  // the head's largest stabiliser: 16-byte loads, eight in flight (nsb % 4 == 0)
+  {
+    const float4* pc4 = reinterpret_cast<const float4*>(pc);
+    const int n4 = P * nsb / 4;
+    for (int i0 = tid; i0 < n4; i0 += 8 * kThreads) {
+      float4 v[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = i0 + u * kThreads < P * nsb ? pc[i0 + u * kThreads] : -INFINITY;
+      for (int u = 0; u < 8; ++u)
+        v[u] = i0 + u * kThreads < n4 ? pc4[i0 + u * kThreads] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) cs = fmaxf(cs, v[u]);
+      for (int u = 0; u < 8; ++u) cs = fmaxf(cs, fmaxf(fmaxf(v[u].x, v[u].y), fmaxf(v[u].z, v[u].w)));
+    }
   }
   float val[NC];
 #pragma unroll
