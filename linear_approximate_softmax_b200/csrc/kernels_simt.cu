@@ -192,6 +192,9 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
   __shared__ __align__(16) __half stage[D + 16][32];
   griddep_launch_dependents();
   griddep_wait();  // the partial state comes from the kernel before this one on the stream
+  // That kernel may still have been writing the partial state while this one was already
+  // resident (programmatic launch), so it is read with loads cached in L2 only (__ldcg), never
+  // through the read-only path, which may serve lines from before the writes.
   const int head = blockIdx.y, tid = threadIdx.x;
   const int fl = tid >> 3, f0 = blockIdx.x * 32, f = f0 + fl;  // feature row (< op_tail)
   const int g = tid & 7;
@@ -202,11 +205,11 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
   auto load = [&](int p0) {  // CB chunks' rows of this feature and their stabilisers, all in flight at once
 #pragma unroll
     for (int b = 0; b < CB; ++b) {
-      cc[b] = live && p0 + b < P ? pc[(p0 + b) * nsb + f / kStabBlock] : -INFINITY;
+      cc[b] = live && p0 + b < P ? __ldcg(pc + (p0 + b) * nsb + f / kStabBlock) : -INFINITY;
 #pragma unroll
       for (int k = 0; k < NC; ++k) {
         const int n = g + 8 * k;
-        x[b][k] = live && p0 + b < P && n < D1 ? rows[static_cast<size_t>(p0 + b) * m * D1 + n] : 0.f;
+        x[b][k] = live && p0 + b < P && n < D1 ? __ldcg(rows + static_cast<size_t>(p0 + b) * m * D1 + n) : 0.f;
       }
     }
   };
@@ -217,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
     for (int p0 = 0; p0 < P; p0 += 8) {
       float v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = p0 + u < P ? pc[(p0 + u) * nsb + f / kStabBlock] : -INFINITY;
+      for (int u = 0; u < 8; ++u) v[u] = p0 + u < P ? __ldcg(pc + (p0 + u) * nsb + f / kStabBlock) : -INFINITY;
 #pragma unroll
       for (int u = 0; u < 8; ++u) cf = fmaxf(cf, v[u]);
     }
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 4 : 2) state_reduce_kernel
       float4 v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        v[u] = i0 + u * kThreads < n4 ? pc4[i0 + u * kThreads] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        v[u] = i0 + u * kThreads < n4 ? __ldcg(pc4 + i0 + u * kThreads) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
 #pragma unroll
       for (int u = 0; u < 8; ++u) cs = fmaxf(cs, fmaxf(fmaxf(v[u].x, v[u].y), fmaxf(v[u].z, v[u].w)));
     }

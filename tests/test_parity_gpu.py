@@ -223,6 +223,27 @@ def test_deterministic_bitwise():
     assert torch.equal(a, b)
 
 
+def test_alternating_shapes_reuse_pool_memory():
+    # Fused calls of two shapes in turn (d = 64 and the multi-query d = 128): each call's scratch
+    # comes back from the stream-ordered pool holding the other shape's partial state and state.
+    # Every kernel must read only what its call wrote, with reads of a preceding kernel's output
+    # that stay coherent while that kernel was still writing (programmatic launches): every
+    # repetition equals the first, bit for bit, and is finite.
+    a = [t.cuda() for t in wl.random_inputs(1, 3, 3, 2000, 64, torch.bfloat16, seed=41)]
+    b = [t.cuda() for t in wl.random_inputs(2, 4, 1, 700, 128, torch.bfloat16, seed=42)]
+    Wa = fv.favor_make_features(5, 256, 64).cuda()
+    Wb = fv.favor_make_features(6, 256, 128).cuda()
+    first = None
+    for it in range(12):
+        oa = fv.favor_attention(*a, Wa)
+        ob = fv.favor_attention(*b, Wb)
+        fv.favor_device_check()
+        assert bool(torch.isfinite(oa).all()) and bool(torch.isfinite(ob).all()), it
+        if first is None:
+            first = (oa.clone(), ob.clone())
+        assert torch.equal(oa, first[0]) and torch.equal(ob, first[1]), it
+
+
 @pytest.mark.parametrize("overlap", [False, True])
 @pytest.mark.parametrize("H,Hkv,d", [(8, 8, 64), (8, 1, 128)])
 def test_back_to_back_calls_reusing_scratch(H, Hkv, d, overlap):
