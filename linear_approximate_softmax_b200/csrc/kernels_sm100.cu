@@ -631,12 +631,14 @@ __global__ void __launch_bounds__(KeyPP<WIDE>::THREADS, 1) key_pass_pp_sm100(
       if (mine > 0) mbar_wait(bar(C::B_SDONE + 2 * w + 1), (mine - 1) & 1, abort_flag, err, 200000000ull);
     }
   } else {
-    // ---------------- key norms: -n(k) = -|k|^2 nscale per token (-inf past the chunk end) ----------------
+    // ---------------- key norms: n(k) = |k|^2 nscale per token (2^100 past the chunk end) ----------------
     // Lane l takes tokens l, l + 32, l + 64, l + 96 of each tile, two at a time.  The 16-byte chunks of a swizzled
     // row are summed in any order; token t starts at chunk t % 8, so the eight lanes of a
-    // shared-memory wavefront hit different banks.  The stage's norms are overwritten only after
-    // the tile that last used it has been contracted, which needs its exponentials, which need
-    // these norms, so no other wait is needed.
+    // shared-memory wavefront hit different banks.  The norms go to the stage's operand of the
+    // projection's norm step (S_NB), read by the tensor cores once the issuer has seen them
+    // published.  The stage's norms are overwritten only after the tile that last used it has
+    // been contracted, which comes after its projection (one thread's MMAs run in issue order),
+    // so no other wait is needed.
     for (int i = 0; i < (RELU ? 0 : ntiles); ++i) {
       const int s = i % C::NST;
       if (!mbar_wait(bar(C::B_KVF + s), (i / C::NST) & 1, abort_flag, err)) break;
