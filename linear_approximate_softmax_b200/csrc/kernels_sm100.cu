@@ -1056,8 +1056,9 @@ struct QueryCfg {
   static constexpr int NSLOT = OWN_SLOT ? 8 : 4;
   static constexpr int S_STG = S_Q + 2 * QTILE;
   static constexpr int S_BAR = S_STG + NSLOT * 32 * 128;
-  static constexpr int B_QF = 0, B_QE = 2, B_CVT = 4, B_UF = 6, B_PHI = 8, B_M2 = 10, B_OF = 12, B_OE = 14,
-                       B_SF = 16, B_SE = 17, B_STG = 18, NBAR = 22;
+  // PHI in halves per warpgroup (2 w + h): phi' of features 64 h .. 64 h + 63 of the block
+  static constexpr int B_QF = 0, B_QE = 2, B_CVT = 4, B_UF = 6, B_PHI = 8, B_M2 = 12, B_OF = 14, B_OE = 16,
+                       B_SF = 18, B_SE = 19, B_STG = 20, NBAR = 24;
   static constexpr int S_TPTR = S_BAR + NBAR * 8;
   static constexpr int S_ABORT = S_TPTR + 8;
   static constexpr int S_IMGS = S_ABORT + 4;  // state images loaded so far (published by warp 3)
@@ -1115,7 +1116,8 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       mbar_init(bar(C::B_QE + i), 1);
       mbar_init(bar(C::B_CVT + i), 4);  // one arrival per epilogue warp
       mbar_init(bar(C::B_UF + i), 1);
-      mbar_init(bar(C::B_PHI + i), 4);
+      mbar_init(bar(C::B_PHI + 2 * i), 4);
+      mbar_init(bar(C::B_PHI + 2 * i + 1), 4);
       mbar_init(bar(C::B_M2 + i), 1);   // the issuer's final drain
       mbar_init(bar(C::B_OF + i), 1);
       mbar_init(bar(C::B_OE + i), 4);
@@ -1280,18 +1282,22 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
       for (int b = 0, tc = 0, j = 0; b < nblk && ok; ++b) {
         const int t = w + 2 * tc, k = cur.img;
         const bool more = b + 1 < nblk, boundary = (j == nb - 1);
-        if (!mbar_wait(bar(C::B_PHI + w), b & 1, abort_flag, err)) break;
         if (j == 0) {
           if (tc >= 1 && !mbar_wait(bar(C::B_OE + w), (tc - 1) & 1, abort_flag, err)) break;
           if (!wait_count_above(img_count, k, abort_flag, err)) break;
         }
-        tc_fence_after();
         const int bw = min(FB, m - FB * j);
-        for (int ks = 0; ks < bw / 16; ++ks) {  // MMA2: O += phi' S', 16 features per step, two per TMEM column
-          const int fk = FB * j + 16 * ks;
-          const uint64_t bd = sdesc_sw128(sbase + C::S_SP + (fk >> 6) * (D * 128) + 32 * ((fk & 63) >> 4), 16, 1024);
-          mma_ts(dO, dU + 8 * ks, bd, id2, (j > 0 || ks > 0) ? 1u : 0u);
+        bool phi_ok = true;
+        for (int h = 0; h < 2 && phi_ok; ++h) {  // MMA2: O += phi' S', each half once its phi' is stored
+          if (!(phi_ok = mbar_wait(bar(C::B_PHI + 2 * w + h), b & 1, abort_flag, err))) break;
+          tc_fence_after();
+          for (int ks = 4 * h; ks < min(4 * h + 4, bw / 16); ++ks) {  // 16 features per step, two per TMEM column
+            const int fk = FB * j + 16 * ks;
+            const uint64_t bd = sdesc_sw128(sbase + C::S_SP + (fk >> 6) * (D * 128) + 32 * ((fk & 63) >> 4), 16, 1024);
+            mma_ts(dO, dU + 8 * ks, bd, id2, (j > 0 || ks > 0) ? 1u : 0u);
+          }
         }
+        if (!phi_ok) break;
         if (boundary) {
           mma_commit(bar(C::B_OF + w));
           TileCursor nx = cur;  // my next tile, t + 2
@@ -1437,12 +1443,14 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
             ph[2 * k4 + 1] = pack_f16x2(p23.x, p23.y);
           }
           tmem_st16(taddr(tbase, eq, cU + 16 * q4), ph);
+          if (q4 & 1) {  // this half's phi' is stored: its contraction steps may go
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::B_PHI + 2 * ewg + (q4 >> 1)));
+          }
         }
         den += den2.x + den2.y;
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::B_PHI + ewg));
       }
       // the tile's blocks are handed over: convert the next tile's Q while the last MMA2 runs
       if (t + 2 < n) up_next = prepare(tc + 1);
