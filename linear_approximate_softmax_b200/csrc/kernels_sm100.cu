@@ -1037,6 +1037,10 @@ struct QueryCfg {
   // warps 4-11 two epilogue warpgroups on alternate tiles
   static constexpr int THREADS = 384;
   static constexpr int EPI0 = 4;
+  // registers after setmaxnreg: producer / MMA / image warpgroup, epilogue warpgroups (the
+  // epilogue holds a 128-feature block of U in registers)
+  static constexpr int R_LOW = 72, R_HIGH = 216;
+  static_assert(128 * R_LOW + 256 * R_HIGH <= 384 * 168, "register split");
   static constexpr int FB = 128;                     // features per block (MMA1 N, MMA2 K)
   static constexpr int MMAX = D == 64 ? 512 : 256;   // features held in shared memory
   static constexpr int QTILE = 128 * D * 2;
@@ -1179,10 +1183,10 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
   const uint32_t tbase = *tptr_slot;
   unsigned int* err = &g_sm100_error_word;
   // registers: the producer / MMA warpgroup gives part of its share to the two epilogue
-  // warpgroups (128 x 88 + 256 x 200 = 62464 <= 384 x 168, the launch allocation; the host
-  // checks the compiled count before launching)
+  // warpgroups (128 x R_LOW + 256 x R_HIGH <= 384 x 168, the launch allocation; the host checks
+  // the compiled count before launching)
   if (warp < C::EPI0) {
-  setmaxnreg_dec<kRegsLow>();
+  setmaxnreg_dec<C::R_LOW>();
   if (warp == 0) {
     // ---------------- producer: Q tiles (stage = tile parity) ----------------
     if (lane == 0) {
@@ -1328,7 +1332,7 @@ __global__ void __launch_bounds__(QueryCfg<D>::THREADS, 1) query_pass_sm100(
     }
   }
   } else {
-    setmaxnreg_inc<kRegsHigh>();
+    setmaxnreg_inc<C::R_HIGH>();
     // ---------------- epilogue warpgroup ewg: tiles ewg, ewg + 2, ... ----------------
     const int eq = warp & 3;
     const int ewg = (warp - C::EPI0) >> 2;
@@ -1626,8 +1630,9 @@ int launch_query(const void* Q, const float* W, const void* state, void* out, co
   if (rc == FAVOR_OK) rc = make_map(&mo, out, D, p.L, bh, 32);  // stored by each epilogue warp, 32 rows
   if (rc != FAVOR_OK) return rc;
   auto kern = query_pass_sm100<D>;
-  static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), C::THREADS);
-  if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), C::THREADS);
+  const long need = 128L * C::R_LOW + 256L * C::R_HIGH;
+  static const int split_ok = check_register_split(reinterpret_cast<const void*>(kern), C::THREADS, need);
+  if (split_ok != FAVOR_OK) return check_register_split(reinterpret_cast<const void*>(kern), C::THREADS, need);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return set_errorf(FAVOR_ERR_CUDA, "sm100 query pass attribute: %s", cudaGetErrorString(e));
   const int ntiles = bh * ((p.L + 127) / 128);
